@@ -1,0 +1,542 @@
+/*
+ * vca_oracle.c -- plain, slow CPU oracle for VC-Attention-style FP8 attention.
+ *
+ * TEST INFRASTRUCTURE ONLY (see vca_oracle.h): used by the tests, the smoke
+ * check and the benchmark's CPU-baseline leg, never by the product path.
+ *
+ * Sources (page titles; sections named where they have one):
+ *   [VCA-news] "VC-Attention: Training-Free Low-Bit Attention Speeds Video
+ *              Diffusion Up to 3.6x" -- V-Smooth and ExpCast-FP8 bullets.
+ *   [VCA-mtp]  "Nunchux AI Introduces VC-Attention: A Training-Free Low-Bit
+ *              Attention Kernel That Speeds Up Video Diffusion Transformers"
+ *              -- Chinese section "V-Smooth 與 ExpCast-FP8" and the English
+ *              abstract ("An E4M3 byte is already close to a logarithm...").
+ *   [VCA-ru]   "VC-Attention" (aikraft.ru) -- section "Решение".
+ *
+ * Where the pages leave a step open, the reading taken is marked READING and
+ * restated in the repository's design notes.
+ */
+#include "vca_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define VO_BLOCK 128
+
+int vo_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------ bf16 */
+
+float vo_bf16_to_float(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* Round a double to the nearest bf16 (8 significant bits), ties to even,
+ * in one step (no intermediate float rounding). */
+uint16_t vo_double_to_bf16_rne(double x) {
+    if (isnan(x)) return 0x7FC0;
+    if (x == 0.0) return signbit(x) ? 0x8000 : 0x0000;
+    double a = fabs(x);
+    int e;
+    frexp(a, &e);                 /* a = f * 2^e, f in [0.5, 1) */
+    int qexp = e - 8;             /* quantum of an 8-significant-bit number */
+    if (qexp < -133) qexp = -133; /* bf16 subnormal quantum 2^-133 */
+    double q = ldexp(a, -qexp);   /* exact (power-of-two scaling) */
+    double r = nearbyint(q);      /* default rounding mode: ties to even */
+    double y = ldexp(r, qexp);    /* exact */
+    float f = (float)y;           /* exact: y has <= 8 significant bits */
+    if (signbit(x)) f = -f;
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);   /* exact: low 16 bits are zero (or inf) */
+}
+
+/* ------------------------------------------------------------------ E4M3 */
+
+/* E4M3 decode from the format's definition: value = (-1)^s * 2^(E-7) * (1+M/8)
+ * for E >= 1, (-1)^s * 2^-6 * (M/8) for E = 0, NaN for E=15,M=7.
+ * ([VCA-mtp]: ExpCast reads this byte, as an integer, as ~8*log2(v)+56.) */
+double vo_e4m3_decode(uint8_t code) {
+    int s = code >> 7, E = (code >> 3) & 15, M = code & 7;
+    double v;
+    if (E == 15 && M == 7) return NAN;
+    if (E == 0) v = ldexp((double)M, -9);
+    else        v = ldexp(1.0 + M / 8.0, E - 7);
+    return s ? -v : v;
+}
+
+/* Table of the 127 non-negative finite E4M3 values in code order (ascending). */
+static double g_e4m3_pos[127];
+static int g_e4m3_init = 0;
+static void e4m3_table_init(void) {
+    if (g_e4m3_init) return;
+    for (int c = 0; c < 127; ++c) g_e4m3_pos[c] = vo_e4m3_decode((uint8_t)c);
+    g_e4m3_init = 1;
+}
+
+/* Nearest E4M3 to x, ties to the even code, finite values saturated to +-448
+ * (READING: saturating conversion; a NaN input gives 0x7F; negative values that
+ * round to zero keep the sign, 0x80). */
+uint8_t vo_e4m3_encode(float x) {
+    e4m3_table_init();
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;
+    /* binary search for the last code with value <= a */
+    int lo = 0, hi = 126;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) / 2;
+        if (g_e4m3_pos[mid] <= a) lo = mid; else hi = mid - 1;
+    }
+    int c = lo;
+    if (c < 126) {
+        double dlo = a - g_e4m3_pos[c], dhi = g_e4m3_pos[c + 1] - a;
+        if (dhi < dlo || (dhi == dlo && ((c + 1) & 1) == 0)) c = c + 1;
+    }
+    return sign | (uint8_t)c;
+}
+
+void vo_e4m3_encode_array(const float* x, uint8_t* out, int64_t n) {
+    e4m3_table_init();
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = vo_e4m3_encode(x[i]);
+}
+
+/* --------------------------------------------------------------- ExpCast */
+
+/* ExpCast-FP8 ([VCA-news] ExpCast-FP8 bullet; [VCA-mtp] abstract; [VCA-ru]
+ * "Решение"): the E4M3 byte of p = 2^z is written straight from z with one
+ * fused multiply-add, byte = 8*z + 56 + beta with beta = -0.35, instead of
+ * computing 2^z in fp32 and casting.
+ * READING: the FMA is fp32 fmaf(8, z, 55.65f); rounding to the byte is
+ * round-to-nearest-even (the pages' 79.6% same-byte rate holds for RNE, not for
+ * truncation); the byte is clamped to [0, 126] (0 = probability 0, 126 = 448,
+ * 127 would be NaN); codes 1..7 are left as computed and decode as E4M3
+ * subnormals (the "underflow tail"); z = NaN gives 0x7F. */
+uint8_t vo_expcast(float z, int flags) {
+    if (isnan(z)) return 0x7F;
+    float addend = (flags & VO_PLANT_BETA0) ? 56.0f : 55.65f;
+    float a = fmaf(8.0f, z, addend);
+    float r = (flags & VO_PLANT_TRUNC) ? floorf(a) : rintf(a);
+    if (r < 0.0f) r = 0.0f;
+    if (r > 126.0f) r = 126.0f;
+    return (uint8_t)r;
+}
+
+void vo_expcast_array(const float* z, uint8_t* out, int64_t n, int flags) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = vo_expcast(z[i], flags);
+}
+
+/* --------------------------------------------------------------- k-means */
+
+/* Squared L2 distance in fp32, channel order 0..d-1, one fmaf per channel.
+ * READING: the pages say only "lightweight k-means" ([VCA-ru] "Решение") /
+ * "lightweight online clustering" ([VCA-news]); this fixed fp32 order makes
+ * the assignment reproducible bit for bit. */
+static float sqdist_f32(const float* v, const float* mu, int d) {
+    float acc = 0.0f;
+    for (int c = 0; c < d; ++c) {
+        float t = v[c] - mu[c];
+        acc = fmaf(t, t, acc);
+    }
+    return acc;
+}
+
+/* Assignment step: each token goes to the centroid at least squared distance;
+ * ties go to the lowest cluster index. */
+void vo_kmeans_assign(const float* v, int N, int d, const float* cent, int k,
+                      int32_t* assign) {
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        const float* x = v + (int64_t)n * d;
+        int best = 0;
+        float bd = sqdist_f32(x, cent, d);
+        for (int c = 1; c < k; ++c) {
+            float dd = sqdist_f32(x, cent + (int64_t)c * d, d);
+            if (dd < bd) { bd = dd; best = c; }
+        }
+        assign[n] = best;
+    }
+}
+
+/* Update step: each centroid becomes the mean of its members.  READING: the
+ * sum is taken exactly in 2^-24 fixed point (int64), so its value does not
+ * depend on summation order; mean = (float)(sum / (count * 2^24)) with one
+ * fp64 division; a cluster with no members keeps its previous centroid. */
+void vo_kmeans_update(const float* v, int N, int d, const int32_t* assign, int k,
+                      float* cent, int32_t* counts) {
+    int64_t* sums = (int64_t*)calloc((size_t)k * d, sizeof(int64_t));
+    for (int c = 0; c < k; ++c) counts[c] = 0;
+    for (int n = 0; n < N; ++n) {
+        int a = assign[n];
+        counts[a] += 1;
+        for (int ch = 0; ch < d; ++ch)
+            sums[(int64_t)a * d + ch] += llrint((double)v[(int64_t)n * d + ch] * 16777216.0);
+    }
+    for (int c = 0; c < k; ++c) {
+        if (counts[c] == 0) continue;
+        double den = (double)counts[c] * 16777216.0;
+        for (int ch = 0; ch < d; ++ch)
+            cent[(int64_t)c * d + ch] = (float)((double)sums[(int64_t)c * d + ch] / den);
+    }
+    free(sums);
+}
+
+/* Lloyd k-means on one head's value tokens.  READING: features are the raw
+ * value vectors; the initial centroid c is token floor(c*N/k) unless warm-start
+ * centroids are given; `iters` rounds of (assign all, then update all); the
+ * returned assignment is the one the final centroids are the means of. */
+void vo_kmeans_head(const uint16_t* V, int N, int d, int k, int iters,
+                    const float* init, float* cent, int32_t* assign, int32_t* counts) {
+    float* v = (float*)malloc((size_t)N * d * sizeof(float));
+    for (int64_t i = 0; i < (int64_t)N * d; ++i) v[i] = vo_bf16_to_float(V[i]);
+    if (init) {
+        memcpy(cent, init, (size_t)k * d * sizeof(float));
+    } else {
+        for (int c = 0; c < k; ++c) {
+            int64_t src = ((int64_t)c * N) / k;
+            memcpy(cent + (int64_t)c * d, v + src * d, (size_t)d * sizeof(float));
+        }
+    }
+    for (int it = 0; it < iters; ++it) {
+        vo_kmeans_assign(v, N, d, cent, k, assign);
+        vo_kmeans_update(v, N, d, assign, k, cent, counts);
+    }
+    free(v);
+}
+
+/* --------------------------------------------------------------- permutation */
+
+/* Tokens reordered by cluster, original order kept inside a cluster
+ * ([VCA-mtp]: the block mean removes more energy "after sorting").
+ * perm[new position] = original index. */
+void vo_stable_perm(const int32_t* assign, int N, int k, int32_t* perm) {
+    int64_t* off = (int64_t*)calloc((size_t)k + 1, sizeof(int64_t));
+    for (int n = 0; n < N; ++n) off[assign[n] + 1] += 1;
+    for (int c = 0; c < k; ++c) off[c + 1] += off[c];
+    for (int n = 0; n < N; ++n) perm[off[assign[n]]++] = n;
+    free(off);
+}
+
+/* --------------------------------------------------------------- quantise */
+
+/* Smallest integer e with amax <= 448 * 2^e (0 for amax = 0), clamped to the
+ * UE8M0 exponent range [-127, 127].  READING: the pages fix no V-residual scale
+ * format; a power of two keeps the rescale exact. */
+int vo_v_exponent(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    int E;
+    double f = frexp((double)amax, &E);   /* amax = f * 2^E, f in [0.5, 1) */
+    /* 448 = 0.875 * 2^9, so amax <= 448*2^e  <=>  f * 2^(E-9-e) <= 0.875 */
+    int e = (f <= 0.875) ? E - 9 : E - 8;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+    return e;
+}
+
+/* Per-block symmetric E4M3 quantisation of 128 token rows (Q in original order,
+ * K in permuted order): scale = amax/448 (fp32), codes = E4M3(x * (448/amax))
+ * with saturation; an all-zero block gets scale 1 and zero codes. */
+static void quant_rows_block(const float* x /* [nv][d] */, int nv, int d,
+                             uint8_t* out /* [128][d] */, float* scale) {
+    float amax = 0.0f;
+    for (int i = 0; i < nv * d; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    memset(out, 0, (size_t)VO_BLOCK * d);
+    if (!(amax > 0.0f)) { *scale = 1.0f; return; }
+    *scale = amax / 448.0f;
+    float inv = 448.0f / amax;
+    for (int i = 0; i < nv * d; ++i) out[i] = vo_e4m3_encode(x[i] * inv);
+}
+
+/* V-Smooth on one head ([VCA-news] V-Smooth bullet; [VCA-ru] "Решение";
+ * [VCA-mtp] 0.125 bit per value element for the mean):
+ *   K and V rows are gathered by the permutation; in each block of 128
+ *   permuted tokens the per-channel mean of V is taken and stored (READING:
+ *   exact fixed-point sum, one fp64 division, rounded once to bf16 -- 16 bits
+ *   per (block, channel) = 0.125 bit per element); only the residual
+ *   r = v - mean (fp32) is quantised to E4M3 with a power-of-two block scale;
+ *   K (permuted) and Q (original order) get per-block fp32 scales. */
+void vo_smooth_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                             const int32_t* perm, int N, int d,
+                             uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                             uint8_t* VrT, int8_t* v_exp, uint16_t* v_mean) {
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    int64_t Np = (int64_t)nb * VO_BLOCK;
+    memset(VrT, 0, (size_t)d * Np);
+#pragma omp parallel for schedule(dynamic)
+    for (int b = 0; b < nb; ++b) {
+        int n0 = b * VO_BLOCK;
+        int nv = N - n0 < VO_BLOCK ? N - n0 : VO_BLOCK;
+        float* xq = (float*)malloc((size_t)VO_BLOCK * d * sizeof(float));
+        float* xk = (float*)malloc((size_t)VO_BLOCK * d * sizeof(float));
+        float* xv = (float*)malloc((size_t)VO_BLOCK * d * sizeof(float));
+        for (int t = 0; t < nv; ++t) {
+            int64_t src = perm[n0 + t];
+            for (int c = 0; c < d; ++c) {
+                xq[t * d + c] = vo_bf16_to_float(Q[(int64_t)(n0 + t) * d + c]);
+                xk[t * d + c] = vo_bf16_to_float(K[src * d + c]);
+                xv[t * d + c] = vo_bf16_to_float(V[src * d + c]);
+            }
+        }
+        quant_rows_block(xq, nv, d, Qq + (int64_t)n0 * d, &q_scale[b]);
+        quant_rows_block(xk, nv, d, Kq + (int64_t)n0 * d, &k_scale[b]);
+        /* V block mean, stored as bf16 */
+        float amax = 0.0f;
+        for (int c = 0; c < d; ++c) {
+            int64_t S = 0;
+            for (int t = 0; t < nv; ++t) S += llrint((double)xv[t * d + c] * 16777216.0);
+            double mean = (double)S / ((double)nv * 16777216.0);
+            uint16_t mb = vo_double_to_bf16_rne(mean);
+            v_mean[(int64_t)b * d + c] = mb;
+            float mf = vo_bf16_to_float(mb);
+            for (int t = 0; t < nv; ++t) {
+                float r = xv[t * d + c] - mf;
+                xv[t * d + c] = r;
+                if (fabsf(r) > amax) amax = fabsf(r);
+            }
+        }
+        int e = vo_v_exponent(amax);
+        v_exp[b] = (int8_t)e;
+        for (int c = 0; c < d; ++c)
+            for (int t = 0; t < nv; ++t)
+                VrT[(int64_t)c * Np + n0 + t] = vo_e4m3_encode(ldexpf(xv[t * d + c], -e));
+        free(xq); free(xk); free(xv);
+    }
+}
+
+/* --------------------------------------------------------------- attention */
+
+/* The ExpCast max grid: m = phi + n with integer n and phi = 0.65/8, so that
+ * 8*(z - m) + 55.65 = 8*z + 55 - 8*n.  READING: snapping the row maximum to
+ * this grid makes any two maxima differ by whole octaves, so the probability
+ * codes computed against a running maximum equal the final ones shifted by a
+ * multiple of 8 (an exact power-of-two rescale). */
+#define VO_PHI (0.65 / 8.0)
+
+/* READING: probabilities are encoded relative to a reference 4 octaves below
+ * the snapped row maximum, i.e. the byte written is ExpCast of z - m + 4: the
+ * row maximum lands on codes 80..88 (p between 8 and 16) instead of 48..56.
+ * This fixed power-of-two pre-scale cancels in the normalisation; it moves the
+ * E4M3 underflow tail 4 octaves further from the maximum and leaves 4 octaves
+ * (codes up to 120 < 126) for a running maximum that lags the true one. */
+#define VO_HEADROOM 4
+
+/* One query row of the same-algorithm attention ([VCA-news] V-Smooth and
+ * ExpCast-FP8 bullets: the block mean is restored from the row sums that
+ * online softmax keeps).  Operands are decoded values in fp64:
+ *   q[d] and its block scale qs; kh[N][d], ks[N] (permuted keys and their
+ *   block scales); rh[N][d] residual codes decoded; vexp[nb]; mu[nb][d].
+ * Steps: s_j = q.k_j; z_j = s_j*qs*ks_j*scale*log2(e); m = snapped max;
+ * p_j = decode(ExpCast code of z_j - m); l_b = sum of p_j over block b;
+ * acc = sum_b 2^vexp_b * sum_{j in b} p_j r_j + sum_b l_b mu_b;
+ * O = acc / sum_b l_b. */
+static void attn_row(const double* q, double qs, const double* kh, const double* ks,
+                     const double* rh, const int* vexp, const double* mu, int N, int d,
+                     double softmax_scale, int flags, double* O, double* lse,
+                     double* lblk, double* z /* scratch [N] */, double* acc /* [d] */) {
+    const double log2e = 1.4426950408889634074;
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    double zmax = -INFINITY;
+    for (int j = 0; j < N; ++j) {
+        double s = 0.0;
+        for (int c = 0; c < d; ++c) s += q[c] * kh[(int64_t)j * d + c];
+        z[j] = s * qs * ks[j] * softmax_scale * log2e;
+        if (z[j] > zmax) zmax = z[j];
+    }
+    double n = ceil(zmax - VO_PHI);
+    for (int c = 0; c < d; ++c) acc[c] = 0.0;
+    double ltot = 0.0;
+    for (int b = 0; b < nb; ++b) {
+        int j0 = b * VO_BLOCK, j1 = j0 + VO_BLOCK < N ? j0 + VO_BLOCK : N;
+        double lb = 0.0;
+        double pv[512];
+        for (int c = 0; c < d; ++c) pv[c] = 0.0;
+        for (int j = j0; j < j1; ++j) {
+            double p;
+            if (flags & VO_EXACT_EXP) {
+                p = exp2(z[j] - (n + VO_PHI) + VO_HEADROOM);
+            } else {
+                /* = 8(z - m) + 55.65 + 8*VO_HEADROOM, m = n + phi */
+                double x = 8.0 * z[j] + 55.0 - 8.0 * n + 8.0 * VO_HEADROOM;
+                if (flags & VO_PLANT_BETA0) x += 0.35;
+                double r = (flags & VO_PLANT_TRUNC) ? floor(x) : nearbyint(x);
+                if (r < 0.0) r = 0.0;
+                if (r > 126.0) r = 126.0;
+                p = vo_e4m3_decode((uint8_t)r);
+            }
+            lb += p;
+            for (int c = 0; c < d; ++c) pv[c] += p * rh[(int64_t)j * d + c];
+        }
+        double sc = ldexp(1.0, vexp[b]);
+        for (int c = 0; c < d; ++c) {
+            acc[c] += sc * pv[c];
+            if (!(flags & VO_PLANT_NO_MEAN)) acc[c] += lb * mu[(int64_t)b * d + c];
+        }
+        if (lblk) lblk[b] = lb;
+        ltot += lb;
+    }
+    for (int c = 0; c < d; ++c) O[c] = acc[c] / ltot;
+    if (lse) *lse = log(2.0) * ((n + VO_PHI - VO_HEADROOM) + log2(ltot));
+}
+
+static void attn_rows(const double* qh, const double* qs_row, const double* kh,
+                      const double* ks, const double* rh, const int* vexp,
+                      const double* mu, int N, int d, double softmax_scale,
+                      const int32_t* rows, int nrows, int flags, double* O,
+                      double* lse, double* lblk) {
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+#pragma omp parallel
+    {
+        double* z = (double*)malloc((size_t)N * sizeof(double));
+        double* acc = (double*)malloc((size_t)d * sizeof(double));
+#pragma omp for schedule(dynamic, 4)
+        for (int r = 0; r < nrows; ++r) {
+            int i = rows[r];
+            attn_row(qh + (int64_t)i * d, qs_row[i], kh, ks, rh, vexp, mu, N, d,
+                     softmax_scale, flags, O + (int64_t)r * d, lse ? &lse[r] : NULL,
+                     lblk ? lblk + (int64_t)r * nb : NULL, z, acc);
+        }
+        free(z);
+        free(acc);
+    }
+}
+
+void vo_attention_head(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                       const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                       const uint16_t* v_mean, int N, int d, double softmax_scale,
+                       const int32_t* rows, int nrows, int flags,
+                       double* O, double* lse, double* lblk) {
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    int64_t Np = (int64_t)nb * VO_BLOCK;
+    double* qh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* kh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* rh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* qs = (double*)malloc((size_t)N * sizeof(double));
+    double* ks = (double*)malloc((size_t)N * sizeof(double));
+    double* mu = (double*)malloc((size_t)nb * d * sizeof(double));
+    int* ve = (int*)malloc((size_t)nb * sizeof(int));
+    for (int j = 0; j < N; ++j) {
+        qs[j] = q_scale[j / VO_BLOCK];
+        ks[j] = k_scale[j / VO_BLOCK];
+        for (int c = 0; c < d; ++c) {
+            qh[(int64_t)j * d + c] = vo_e4m3_decode(Qq[(int64_t)j * d + c]);
+            kh[(int64_t)j * d + c] = vo_e4m3_decode(Kq[(int64_t)j * d + c]);
+            rh[(int64_t)j * d + c] = vo_e4m3_decode(VrT[(int64_t)c * Np + j]);
+        }
+    }
+    for (int b = 0; b < nb; ++b) {
+        ve[b] = v_exp[b];
+        for (int c = 0; c < d; ++c) mu[(int64_t)b * d + c] = vo_bf16_to_float(v_mean[(int64_t)b * d + c]);
+    }
+    attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, O, lse, lblk);
+    free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
+}
+
+void vo_attention_head_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                            const int32_t* perm, int N, int d, double softmax_scale,
+                            const int32_t* rows, int nrows, int flags, double* O) {
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    int64_t Np = (int64_t)nb * VO_BLOCK;
+    if (!(flags & VO_IDENTITY_QUANT)) {
+        uint8_t* Qq = (uint8_t*)malloc((size_t)Np * d);
+        uint8_t* Kq = (uint8_t*)malloc((size_t)Np * d);
+        uint8_t* VrT = (uint8_t*)malloc((size_t)Np * d);
+        float* qsc = (float*)malloc((size_t)nb * sizeof(float));
+        float* ksc = (float*)malloc((size_t)nb * sizeof(float));
+        int8_t* ve = (int8_t*)malloc((size_t)nb);
+        uint16_t* vm = (uint16_t*)malloc((size_t)nb * d * sizeof(uint16_t));
+        vo_smooth_quantize_head(Q, K, V, perm, N, d, Qq, qsc, Kq, ksc, VrT, ve, vm);
+        vo_attention_head(Qq, qsc, Kq, ksc, VrT, ve, vm, N, d, softmax_scale, rows, nrows,
+                          flags, O, NULL, NULL);
+        free(Qq); free(Kq); free(VrT); free(qsc); free(ksc); free(ve); free(vm);
+        return;
+    }
+    /* Identity quantisers: operands kept exactly, block means exact in fp64. */
+    double* qh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* kh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* rh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* ones = (double*)malloc((size_t)N * sizeof(double));
+    double* mu = (double*)malloc((size_t)nb * d * sizeof(double));
+    int* ve = (int*)calloc((size_t)nb, sizeof(int));
+    for (int j = 0; j < N; ++j) {
+        ones[j] = 1.0;
+        for (int c = 0; c < d; ++c) {
+            qh[(int64_t)j * d + c] = vo_bf16_to_float(Q[(int64_t)j * d + c]);
+            kh[(int64_t)j * d + c] = vo_bf16_to_float(K[(int64_t)perm[j] * d + c]);
+            rh[(int64_t)j * d + c] = vo_bf16_to_float(V[(int64_t)perm[j] * d + c]);
+        }
+    }
+    for (int b = 0; b < nb; ++b) {
+        int j0 = b * VO_BLOCK, j1 = j0 + VO_BLOCK < N ? j0 + VO_BLOCK : N;
+        for (int c = 0; c < d; ++c) {
+            double s = 0.0;
+            for (int j = j0; j < j1; ++j) s += rh[(int64_t)j * d + c];
+            double m = s / (j1 - j0);
+            mu[(int64_t)b * d + c] = m;
+            for (int j = j0; j < j1; ++j) rh[(int64_t)j * d + c] -= m;
+        }
+    }
+    attn_rows(qh, ones, kh, ones, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, O,
+              NULL, NULL);
+    free(qh); free(kh); free(rh); free(ones); free(mu); free(ve);
+}
+
+/* Exact softmax attention in fp64, two passes (max, then sum) per row. */
+void vo_exact_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                             int N, int d, double softmax_scale,
+                             const int32_t* rows, int nrows, double* O) {
+    double* kd = (double*)malloc((size_t)N * d * sizeof(double));
+    double* vd = (double*)malloc((size_t)N * d * sizeof(double));
+    for (int64_t i = 0; i < (int64_t)N * d; ++i) {
+        kd[i] = vo_bf16_to_float(K[i]);
+        vd[i] = vo_bf16_to_float(V[i]);
+    }
+#pragma omp parallel
+    {
+        double* a = (double*)malloc((size_t)N * sizeof(double));
+        double* q = (double*)malloc((size_t)d * sizeof(double));
+#pragma omp for schedule(dynamic, 4)
+        for (int r = 0; r < nrows; ++r) {
+            int i = rows[r];
+            for (int c = 0; c < d; ++c) q[c] = vo_bf16_to_float(Q[(int64_t)i * d + c]);
+            double m = -INFINITY;
+            for (int j = 0; j < N; ++j) {
+                double s = 0.0;
+                for (int c = 0; c < d; ++c) s += q[c] * kd[(int64_t)j * d + c];
+                a[j] = s * softmax_scale;
+                if (a[j] > m) m = a[j];
+            }
+            double l = 0.0;
+            double* o = O + (int64_t)r * d;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            for (int j = 0; j < N; ++j) {
+                double p = exp(a[j] - m);
+                l += p;
+                for (int c = 0; c < d; ++c) o[c] += p * vd[(int64_t)j * d + c];
+            }
+            for (int c = 0; c < d; ++c) o[c] /= l;
+        }
+        free(a);
+        free(q);
+    }
+    free(kd);
+    free(vd);
+}

@@ -1,0 +1,102 @@
+/*
+ * vca_oracle.h -- plain, slow CPU oracle for VC-Attention-style FP8 attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call this
+ * library: only the test suite, the package's smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or constant with
+ * the CUDA library; it is written from the method's description on these pages:
+ *
+ *   [VCA-news] "VC-Attention: Training-Free Low-Bit Attention Speeds Video
+ *              Diffusion Up to 3.6x" (agihunt.info news summary).
+ *   [VCA-mtp]  "Nunchux AI Introduces VC-Attention: A Training-Free Low-Bit
+ *              Attention Kernel That Speeds Up Video Diffusion Transformers"
+ *              (MarkTechPost abstract, mirrored with a Chinese summary on
+ *              yifor-blog; sections "V-Smooth 與 ExpCast-FP8" and the English
+ *              abstract).
+ *   [VCA-ru]   "VC-Attention" (aikraft.ru news), section "Решение:
+ *              VC-Attention без дообучения".
+ *
+ * Arithmetic: fp64 wherever the method does not fix a precision; fp32 with
+ * explicit fmaf() where the method (or a stated reading of it) fixes fp32.
+ * Build with -O2 -ffp-contract=off and no fast-math.
+ *
+ * bf16 tensors are passed as their raw uint16 bit patterns.
+ * All per-head arrays are row-major: [N][d] for token rows, [d][Np] for the
+ * transposed V residual, [nb][d] for block means.
+ */
+#ifndef VCA_ORACLE_H
+#define VCA_ORACLE_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- flags for vo_attention_* (reductions and planted mistakes) ---- */
+#define VO_EXACT_EXP       1   /* p = 2^(z - m) in fp64 instead of ExpCast codes     */
+#define VO_IDENTITY_QUANT  2   /* bf16 path only: no E4M3 rounding, exact fp64 means  */
+#define VO_PLANT_TRUNC     64  /* planted mistake: ExpCast truncates instead of RNE  */
+#define VO_PLANT_NO_MEAN   128 /* planted mistake: drop the rowsum*mean restore term */
+#define VO_PLANT_BETA0     256 /* planted mistake: addend 56 instead of 56 + beta    */
+
+/* E4M3 (OCP FP8: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
+ * no infinities, NaN = S.1111.111, largest finite 448). */
+double  vo_e4m3_decode(uint8_t code);
+uint8_t vo_e4m3_encode(float x);
+void    vo_e4m3_encode_array(const float* x, uint8_t* out, int64_t n);
+
+/* ExpCast-FP8 on a log2-domain, max-subtracted score z. */
+uint8_t vo_expcast(float z, int flags);
+void    vo_expcast_array(const float* z, uint8_t* out, int64_t n, int flags);
+
+/* bf16 helpers. */
+float    vo_bf16_to_float(uint16_t b);
+uint16_t vo_double_to_bf16_rne(double x);
+
+/* k-means over the value tokens of one head. */
+void vo_kmeans_assign(const float* v, int N, int d, const float* cent, int k,
+                      int32_t* assign);
+void vo_kmeans_update(const float* v, int N, int d, const int32_t* assign, int k,
+                      float* cent, int32_t* counts);
+void vo_kmeans_head(const uint16_t* V, int N, int d, int k, int iters,
+                    const float* init /* nullable [k][d] */, float* cent /* [k][d] */,
+                    int32_t* assign /* [N] */, int32_t* counts /* [k] */);
+
+/* Stable counting sort by cluster id: perm[new] = old. */
+void vo_stable_perm(const int32_t* assign, int N, int k, int32_t* perm);
+
+/* V-Smooth quantisation of one head (block = 128 tokens, Np = 128*ceil(N/128)). */
+int  vo_v_exponent(float amax);
+void vo_smooth_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                             const int32_t* perm, int N, int d,
+                             uint8_t* Qq /* [Np][d] */, float* q_scale /* [nb] */,
+                             uint8_t* Kq /* [Np][d] */, float* k_scale /* [nb] */,
+                             uint8_t* VrT /* [d][Np] */, int8_t* v_exp /* [nb] */,
+                             uint16_t* v_mean /* [nb][d] */);
+
+/* Same-algorithm attention for selected query rows of one head, from the
+ * quantised operands.  O is [nrows][d] fp64, lse [nrows] (nullable),
+ * lblk [nrows][nb] per-block row sums (nullable). */
+void vo_attention_head(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                       const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                       const uint16_t* v_mean, int N, int d, double softmax_scale,
+                       const int32_t* rows, int nrows, int flags,
+                       double* O, double* lse, double* lblk);
+
+/* Same algorithm, straight from bf16 Q/K/V and a permutation; with
+ * VO_IDENTITY_QUANT the quantisers are the identity (for reductions). */
+void vo_attention_head_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                            const int32_t* perm, int N, int d, double softmax_scale,
+                            const int32_t* rows, int nrows, int flags, double* O);
+
+/* Exact fp64 softmax(Q K^T * scale) V for selected rows of one head. */
+void vo_exact_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                             int N, int d, double softmax_scale,
+                             const int32_t* rows, int nrows, double* O);
+
+int vo_num_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
