@@ -1,0 +1,471 @@
+// vca_attn_fp8.cu -- ExpCast-FP8 flash attention with V-Smooth mean restore.
+//
+// Method ("VC-Attention: Training-Free Low-Bit Attention Speeds Video
+// Diffusion Up to 3.6x", V-Smooth and ExpCast-FP8 bullets; "Nunchux AI
+// Introduces VC-Attention..." abstract; "VC-Attention", aikraft.ru, "Решение"):
+// QK^T and PV run on 8-bit tensor cores; the softmax writes each E4M3
+// probability byte from the log-domain score with one FMA (byte ~ 8 log2 p + 56
+// + beta, beta = -0.35) instead of an fp32 exp2 and a cast; the value block
+// mean that prep subtracted is restored from the per-block row sums.
+//
+// Design (sm_100a):
+//  * one CTA = two 128-row query tiles of one head (they share every K/V tile);
+//    12 warps: warp 0 TMA producer, warp 1 MMA issuer (one thread) and TMEM
+//    owner, warp 2 stages block means, warps 4-7 / 8-11 are the softmax
+//    warpgroups of query tile 0 / 1 (thread = query row = TMEM lane).
+//  * TMEM (512 columns): S0, S1 (fp32 scores), O0, O1 (fp32 accumulators).
+//  * S_t = Q_t K_j^T: tcgen05 kind::f8f6f4, operands from 128B-swizzled smem.
+//  * O_t += P_t R_j * 2^e_j: kind::mxf8f6f4.block_scale; the per-block V
+//    exponent is the UE8M0 scale of B (A's scale is 1).  The two 4-column scale
+//    vectors are written into the already-consumed S_t columns, so the next
+//    QK^T (issued after this PV, and tensor-core ops run in issue order)
+//    overwrites them only after they were read.
+//  * Mean restore: every 8 key blocks, O_t += L_t M^T with a TF32 MMA, where
+//    L_t[i][b] are the block row sums (split hi + lo so they keep ~22 bits) and
+//    M[d][b] the bf16 block means (exact in TF32).
+//  * Online maximum on the grid phi + integers (phi = 0.65/8): a lagging
+//    maximum changes codes by multiples of 8, i.e. probabilities by exact
+//    powers of two, and O is rescaled by exact powers of two only when the
+//    block maximum overtakes the reference by more than 4 octaves.  Codes are
+//    written 4 octaves above the reference (row max at codes 80..88), keeping
+//    the largest code at 120 < 126.
+//  * Every mbarrier wait is bounded (globaltimer); on expiry the CTA records
+//    VCA_ERR_TIMEOUT in the status word, all roles drain and exit, and TMEM is
+//    freed after the issued MMAs complete.
+#include "vca_device.cuh"
+#include "vca_host.h"
+
+namespace vca {
+
+constexpr int kAttnThreads = 384;
+constexpr int kStages = 3;
+constexpr int kGroup = 8;   // key blocks per mean-restore MMA
+
+// dynamic shared memory layout (offsets from a 1024-aligned base)
+constexpr uint32_t kOffQ = 0;                         // 2 x 16 KB
+constexpr uint32_t kOffK = 32768;                     // kStages x 16 KB
+constexpr uint32_t kOffV = kOffK + kStages * 16384;   // kStages x 16 KB
+constexpr uint32_t kOffP = kOffV + kStages * 16384;   // 2 x 16 KB
+constexpr uint32_t kOffL = kOffP + 32768;             // 2 tiles x (hi 4 KB + lo 4 KB)
+constexpr uint32_t kOffMu = kOffL + 16384;            // 2 buffers x 4 KB
+constexpr uint32_t kSmemBytes = kOffMu + 8192;
+constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
+
+struct AttnParams {
+  CUtensorMap tmQ, tmK, tmV;
+  const float* q_scale;
+  const float* k_scale;
+  const int8_t* v_exp;
+  const uint16_t* v_mean;
+  uint16_t* O;
+  float* lse;
+  int N, nb;
+  float c_base;            // softmax_scale * log2(e)
+  DevStatus* st;
+  unsigned long long wait_ns;
+};
+
+struct __align__(8) AttnBars {
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_done[2];
+  uint64_t mu_full[2];
+  uint64_t mu_empty[2];
+  uint64_t mma_done;
+};
+
+// offset of fp32 element (row r, col k) in a K-major, no-swizzle [128 x 8] tile
+__device__ __forceinline__ uint32_t tf32_tile_off(int r, int k) {
+  return (uint32_t)((r >> 3) * 256 + (k >> 2) * 128 + (r & 7) * 16 + (k & 3) * 4);
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_constant__ AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ AttnBars bars;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  __shared__ int never_s;   // abort flag for drain waits: these must not give up early
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = blockIdx.x, bh = blockIdx.y;
+  const int N = p.N, nb = p.nb, nkv = nb;
+  const int ngroups = (nkv + kGroup - 1) / kGroup;
+  const int64_t Np = (int64_t)nb * 128;
+  const uint64_t lim = p.wait_ns;
+
+  if (threadIdx.x == 0) {
+    abort_s = 0;
+    never_s = 0;
+    mbar_init(&bars.q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars.kv_full[s], 1);
+      mbar_init(&bars.kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars.s_full[t], 1);
+      mbar_init(&bars.p_full[t], 128);
+      mbar_init(&bars.o_done[t], 1);
+      mbar_init(&bars.mu_full[t], 32);
+      mbar_init(&bars.mu_empty[t], 1);
+    }
+    mbar_init(&bars.mma_done, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&p.tmQ);
+    tma_prefetch_desc(&p.tmK);
+    tma_prefetch_desc(&p.tmV);
+  }
+  // a CTA of this launch (or of an earlier one sharing the workspace) already
+  // timed out: do no work, so a broken pipeline costs one wait, not one per CTA
+  __shared__ int skip_s;
+  if (threadIdx.x == 0) skip_s = (p.st && *reinterpret_cast<volatile int*>(&p.st->code) == VCA_ERR_TIMEOUT);
+  __syncthreads();
+  if (skip_s) return;
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_s, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars.q_full, 32768);
+      const int qrow = (int)((int64_t)bh * Np) + pair * 256;
+      tma_load_2d(sm + kOffQ, &p.tmQ, &bars.q_full, 0, qrow);
+      tma_load_2d(sm + kOffQ + 16384, &p.tmQ, &bars.q_full, 0, qrow + 128);
+      int issued = 0;
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % kStages, u = j / kStages;
+        if (u > 0 && !mbar_wait_bounded(&bars.kv_empty[s], (u - 1) & 1, &abort_s, p.st, lim, 100)) break;
+        mbar_arrive_expect_tx(&bars.kv_full[s], 32768);
+        tma_load_2d(sm + kOffK + s * 16384, &p.tmK, &bars.kv_full[s], 0, (int)((int64_t)bh * Np) + j * 128);
+        tma_load_2d(sm + kOffV + s * 16384, &p.tmV, &bars.kv_full[s], j * 128, bh * 128);
+        issued = j + 1;
+      }
+      if (abort_s) {
+        // let the copies already issued land before the CTA exits
+        for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j)
+          mbar_wait_bounded(&bars.kv_full[j % kStages], (j / kStages) & 1, &never_s, nullptr, lim, 101);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_qk = instr_desc(kFmtE4M3, kFmtE4M3, 128, 128, 0, 0);
+      const uint32_t id_pv = instr_desc_mx(kFmtE4M3, kFmtE4M3, 128, 128);
+      const uint32_t id_mu = instr_desc(kFmtTF32, kFmtTF32, 128, 128, 0, 0);
+      const uint32_t sQ = smem_u32(sm + kOffQ), sK = smem_u32(sm + kOffK), sV = smem_u32(sm + kOffV);
+      const uint32_t sP = smem_u32(sm + kOffP), sL = smem_u32(sm + kOffL), sMu = smem_u32(sm + kOffMu);
+      bool ok = mbar_wait_bounded(&bars.q_full, 0, &abort_s, p.st, lim, 200);
+      ok = ok && mbar_wait_bounded(&bars.kv_full[0], 0, &abort_s, p.st, lim, 201);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t) {
+          for (int k = 0; k < 4; ++k)
+            mma_f8_ss(tmem + t * 128, smem_desc(sQ + t * 16384 + 32 * k, 16, 1024, kLayoutSW128),
+                      smem_desc(sK + 32 * k, 16, 1024, kLayoutSW128), id_qk, k > 0);
+          tc_commit(&bars.s_full[t]);
+        }
+      }
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int s = j % kStages;
+        const bool group_end = (j % kGroup == kGroup - 1) || (j == nkv - 1);
+        const int g = j / kGroup, gb = g & 1;
+        for (int t = 0; t < 2 && ok; ++t) {
+          ok = mbar_wait_bounded(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t sft = tmem + t * 128;   // scale vectors live in the consumed S_t columns
+          for (int k = 0; k < 4; ++k)
+            mma_mxf8_ss(tmem + 256 + t * 128, smem_desc(sP + t * 16384 + 32 * k, 16, 1024, kLayoutSW128),
+                        smem_desc(sV + s * 16384 + 32 * k, 16, 1024, kLayoutSW128), id_pv, sft, sft + 4,
+                        (j > 0 || k > 0) ? 1u : 0u);
+          if (group_end) {
+            ok = mbar_wait_bounded(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220);
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t bdesc = smem_desc(sMu + gb * 4096, 128, 256, kLayoutNone);
+            mma_tf32_ss(tmem + 256 + t * 128, smem_desc(sL + t * 8192, 128, 256, kLayoutNone), bdesc, id_mu, 1u);
+            mma_tf32_ss(tmem + 256 + t * 128, smem_desc(sL + t * 8192 + 4096, 128, 256, kLayoutNone), bdesc,
+                        id_mu, 1u);
+            if (t == 1) tc_commit(&bars.mu_empty[gb]);
+          }
+          tc_commit(&bars.o_done[t]);
+          if (t == 1) tc_commit(&bars.kv_empty[s]);
+          if (j + 1 < nkv) {
+            const int s1 = (j + 1) % kStages;
+            if (t == 0) {
+              ok = mbar_wait_bounded(&bars.kv_full[s1], ((j + 1) / kStages) & 1, &abort_s, p.st, lim, 230);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            for (int k = 0; k < 4; ++k)
+              mma_f8_ss(tmem + t * 128, smem_desc(sQ + t * 16384 + 32 * k, 16, 1024, kLayoutSW128),
+                        smem_desc(sK + s1 * 16384 + 32 * k, 16, 1024, kLayoutSW128), id_qk, k > 0);
+            tc_commit(&bars.s_full[t]);
+          }
+        }
+      }
+      tc_commit(&bars.mma_done);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ block means -> fp32 [d][8] tiles
+    const uint16_t* vm = p.v_mean + (int64_t)bh * nb * 128;
+    for (int g = 0; g < ngroups; ++g) {
+      const int gb = g & 1, u = g >> 1;
+      if (u > 0 && !mbar_wait_bounded(&bars.mu_empty[gb], (u - 1) & 1, &abort_s, p.st, lim, 300)) break;
+      uint8_t* dst = sm + kOffMu + gb * 4096;
+      for (int q = 0; q < 4; ++q) {
+        const int dch = q * 32 + lane;
+        for (int kk = 0; kk < kGroup; ++kk) {
+          const int blk = g * kGroup + kk;
+          float v = blk < nb ? __uint_as_float((uint32_t)__ldg(vm + (int64_t)blk * 128 + dch) << 16) : 0.0f;
+          *reinterpret_cast<float*>(dst + tf32_tile_off(dch, kk)) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars.mu_full[gb]);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = (warp >> 2) - 1;                 // query tile of this warpgroup
+    const int r = threadIdx.x & 127;               // query row within the tile = TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + t * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + t * 128 + lane_off;
+    const int qtile = pair * 2 + t;
+    const bool qvalid = qtile < nb;
+    const float sq = qvalid ? __ldg(p.q_scale + (int64_t)bh * nb + qtile) : 1.0f;
+    const float cq = sq * p.c_base;
+    const float kMagic = 12582912.0f;              // 1.5 * 2^23: adding it rounds to an integer
+    uint8_t* sP = sm + kOffP + t * 16384;
+    uint8_t* sLt = sm + kOffL + t * 8192;
+    const float* ksc = p.k_scale + (int64_t)bh * nb;
+    const int8_t* vex = p.v_exp + (int64_t)bh * nb;
+    int nref = 0;
+    bool have_ref = false;
+    float ltot = 0.0f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      ok = mbar_wait_warp(&bars.s_full[t], j & 1, &abort_s, p.st, lim, 400 + t);
+      if (!ok) break;
+      tc_fence_after();
+      float sv[128];
+      {
+        uint32_t* su = reinterpret_cast<uint32_t*>(sv);
+        VCA_TMEM_LD32(tS + 0, (su + 0));
+        VCA_TMEM_LD32(tS + 32, (su + 32));
+        VCA_TMEM_LD32(tS + 64, (su + 64));
+        VCA_TMEM_LD32(tS + 96, (su + 96));
+        tmem_ld_wait();
+      }
+      const int valid = min(128, N - j * 128);
+      if (valid < 128) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) sv[c] = -INFINITY;
+      }
+      float mx = sv[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
+      const float cz = cq * __ldg(ksc + j);        // z = s * cz (log2 domain)
+      const float c8 = 8.0f * cz;
+      const int ntile = (int)ceilf(__fmaf_rn(mx, cz, -0.08125f));
+      // the previous PV into O_t (and sP_t, sL_t reads) must be complete before
+      // O_t is rescaled or sP_t / sL_t are overwritten
+      if (j > 0) {
+        ok = mbar_wait_warp(&bars.o_done[t], (j - 1) & 1, &abort_s, p.st, lim, 410 + t);
+        if (!ok) break;
+        tc_fence_after();
+      }
+      float rescale = 1.0f;       // O_t and the pending row sums are scaled by this
+      if (!have_ref) {
+        nref = ntile;
+        have_ref = true;
+      } else if (ntile > nref + 4) {
+        const int delta = ntile - nref;
+        nref = ntile;
+        rescale = delta > 126 ? 0.0f : __uint_as_float((uint32_t)(127 - delta) << 23);
+      }
+      // ExpCast: code = rne(s*c8 + 87 - 8*nref) via the magic-number FMA,
+      // clamped below at 0; p = decode(code) summed exactly as
+      // float(code << 20) * 2^120.
+      const float badd = kMagic + (float)(87 - 8 * nref);
+      float lsum = 0.0f;
+      const uint32_t prow = smem_u32(sP) + r * 128;
+#pragma unroll
+      for (int u16 = 0; u16 < 8; ++u16) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t b[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float f = fmaxf(__fmaf_rn(sv[u16 * 16 + q * 4 + e], c8, badd), kMagic);
+            b[e] = __float_as_uint(f);
+            lsum += __uint_as_float(b[e] << 20);
+          }
+          w4[q] = prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
+        }
+        const uint32_t addr = prow + ((uint32_t)(u16 ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w4[0]), "r"(w4[1]),
+                     "r"(w4[2]), "r"(w4[3])
+                     : "memory");
+      }
+      const float l = lsum * 0x1p120f;
+      // block row sum -> L tile (hi part exact in TF32, lo the remainder)
+      {
+        const int kk = j % kGroup;
+        const float hi = __uint_as_float(__float_as_uint(l) & 0xFFFFE000u);
+        const float lo = l - hi;
+        *reinterpret_cast<float*>(sLt + tf32_tile_off(r, kk)) = hi;
+        *reinterpret_cast<float*>(sLt + 4096 + tf32_tile_off(r, kk)) = lo;
+        if (j == nkv - 1) {
+          for (int k2 = kk + 1; k2 < kGroup; ++k2) {
+            *reinterpret_cast<float*>(sLt + tf32_tile_off(r, k2)) = 0.0f;
+            *reinterpret_cast<float*>(sLt + 4096 + tf32_tile_off(r, k2)) = 0.0f;
+          }
+        }
+      }
+      // tcgen05.ld/st are warp-collective: if any row of the warp rescales, the
+      // whole warp runs the read-modify-write (other rows multiply by 1)
+      if (__any_sync(0xffffffffu, rescale != 1.0f)) {
+        // the reference maximum moved up: O_t and this group's earlier row sums
+        // are scaled by the same exact power of two (S is no longer live here)
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t o[32];
+          VCA_TMEM_LD32(tO + c0, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * rescale);
+          VCA_TMEM_ST32(tO + c0, o);
+        }
+        for (int kk = 0; kk < (j % kGroup); ++kk) {
+          float* hi = reinterpret_cast<float*>(sLt + tf32_tile_off(r, kk));
+          float* lo = reinterpret_cast<float*>(sLt + 4096 + tf32_tile_off(r, kk));
+          *hi *= rescale;
+          *lo *= rescale;
+        }
+      }
+      ltot = ltot * rescale + l;
+      // UE8M0 scale vectors for this PV: A = 2^0, B = 2^v_exp[j]
+      {
+        const uint32_t eb = (uint32_t)(127 + (int)__ldg(vex + j));
+        uint32_t sf[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sf[i] = 0x7F7F7F7Fu;
+#pragma unroll
+        for (int i = 4; i < 8; ++i) sf[i] = eb * 0x01010101u;
+        tmem_st8(tS, sf);
+      }
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars.p_full[t]);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = mbar_wait_warp(&bars.o_done[t], (nkv - 1) & 1, &abort_s, p.st, lim, 420 + t);
+    if (ok) {
+      tc_fence_after();
+      const int qrow = qtile * 128 + r;
+      const bool store = qvalid && qrow < N;
+      const float inv = 1.0f / ltot;
+      uint16_t* orow = p.O + ((int64_t)bh * N + qrow) * 128;
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t o[32];
+        VCA_TMEM_LD32(tO + c0, o);
+        tmem_ld_wait();
+        if (store) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[2 * c]) * inv,
+                                                     __uint_as_float(o[2 * c + 1]) * inv);
+            pk[c] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+      }
+      if (store && p.lse)
+        p.lse[(int64_t)bh * N + qrow] = 0.69314718055994531f * ((float)nref + 0.08125f - 4.0f + __log2f(ltot));
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    // every issued MMA has completed before TMEM is released
+    mbar_wait_bounded(&bars.mma_done, 0, &never_s, nullptr, lim, 500);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace vca
+
+using namespace vca;
+
+extern "C" size_t vca_attention_workspace_size(int B, int H, int N) { return 256; }
+
+extern "C" int vca_attention_fwd(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                                 const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                                 const vca_bf16* v_mean, int B, int H, int N, int d,
+                                 float softmax_scale, vca_bf16* O, float* lse, void* ws,
+                                 size_t ws_bytes, vca_stream_t stream) {
+  if (d != VCA_HEAD_DIM) return fail(VCA_ERR_UNSUPPORTED, "vca_attention_fwd: d must be 128");
+  if (B < 1 || H < 1 || N < 1 || (int64_t)B * H > 65535)
+    return fail(VCA_ERR_INVALID, "vca_attention_fwd: bad shape B=%d H=%d N=%d", B, H, N);
+  const int nb = (N + 127) / 128;
+  const int64_t Np = (int64_t)nb * 128;
+  if ((int64_t)B * H * Np > INT32_MAX || Np > INT32_MAX / 2)
+    return fail(VCA_ERR_UNSUPPORTED, "vca_attention_fwd: B*H*Np exceeds the 2^31 row limit");
+  const void* ptrs[] = {Qq, q_scale, Kq, k_scale, VrT, v_exp, v_mean, O};
+  for (const void* q : ptrs)
+    if (!q) return fail(VCA_ERR_INVALID, "vca_attention_fwd: null pointer");
+  const void* al[] = {Qq, Kq, VrT, O};
+  for (const void* q : al)
+    if (!aligned16(q)) return fail(VCA_ERR_INVALID, "vca_attention_fwd: tensors must be 16-byte aligned");
+  if (!(softmax_scale > 0.0f)) return fail(VCA_ERR_INVALID, "vca_attention_fwd: softmax_scale must be > 0");
+  if (!ws || ws_bytes < vca_attention_workspace_size(B, H, N))
+    return fail(VCA_ERR_WORKSPACE, "vca_attention_fwd: workspace too small");
+
+  AttnParams prm;
+  const uint64_t BH = (uint64_t)B * H;
+  {
+    uint64_t dims[2] = {128, BH * (uint64_t)Np}, str[1] = {128};
+    uint32_t box[2] = {128, 128};
+    int rc = encode_tiled(&prm.tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Qq, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!rc) rc = encode_tiled(&prm.tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, Kq, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    uint64_t vd[2] = {(uint64_t)Np, BH * 128}, vs[1] = {(uint64_t)Np};
+    if (!rc) rc = encode_tiled(&prm.tmV, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, VrT, vd, vs, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+  }
+  prm.q_scale = q_scale;
+  prm.k_scale = k_scale;
+  prm.v_exp = v_exp;
+  prm.v_mean = v_mean;
+  prm.O = O;
+  prm.lse = lse;
+  prm.N = N;
+  prm.nb = nb;
+  prm.c_base = (float)((double)softmax_scale * 1.4426950408889634);
+  prm.st = (DevStatus*)ws;
+  prm.wait_ns = wait_limit_ns();
+  if (cudaFuncSetAttribute(attn_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc) !=
+      cudaSuccess)
+    return fail(VCA_ERR_CUDA, "vca_attention_fwd: cannot set shared-memory size");
+  dim3 grid((nb + 1) / 2, (unsigned)BH);
+  attn_fp8_kernel<<<grid, kAttnThreads, kSmemAlloc, (cudaStream_t)stream>>>(prm);
+  return check_launch("attn_fp8_kernel");
+}

@@ -1,0 +1,303 @@
+// vca_kmeans.cu -- V-Smooth grouping: k-means over value tokens and the stable
+// permutation that sorts tokens by cluster.
+//
+// Method: "VC-Attention: Training-Free Low-Bit Attention Speeds Video Diffusion
+// Up to 3.6x" (V-Smooth bullet): value tokens are reordered by lightweight
+// online clustering so a hardware block holds tokens that quantise well
+// together; "VC-Attention" (aikraft.ru, section "Решение"): a lightweight
+// k-means groups similar tokens into blocks; "Nunchux AI Introduces
+// VC-Attention..." (abstract): the block mean removes far more energy after
+// sorting.
+//
+// Per round: assign (token-parallel; fp32 distances in channel order, one FMA
+// per channel, so the argmin is reproducible bit for bit), accumulate
+// (channel-parallel exact 2^-24 fixed-point sums in int64, order-free), update
+// (one fp64 division per centroid coordinate).  Then a stable counting sort:
+// per-chunk histograms, an exclusive scan in (cluster, chunk) order, and a
+// warp-synchronous ranked scatter.
+#include "vca_device.cuh"
+#include "vca_host.h"
+
+namespace vca {
+
+constexpr int kAssignThreads = 128;
+constexpr int kAccumChunk = 2048;   // tokens per accumulate CTA
+constexpr int kSortChunk = 1024;    // tokens per sort CTA
+
+struct KmWs {
+  DevStatus* st;
+  long long* sums;   // [BH][k][128]
+  int* counts;       // [BH][k]
+  int* ccount;       // [BH][nchunk][k]  per-chunk histogram
+  int* cbase;        // [BH][nchunk][k]  scatter base per (chunk, cluster)
+};
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static KmWs carve(void* ws, int BH, int N, int k, size_t* total) {
+  size_t nchunk = (size_t)(N + kSortChunk - 1) / kSortChunk;
+  size_t off = 0;
+  KmWs w;
+  char* base = (char*)ws;
+  w.st = (DevStatus*)(base + off);
+  off += 256;
+  w.sums = (long long*)(base + off);
+  off += align256((size_t)BH * k * 128 * sizeof(long long));
+  w.counts = (int*)(base + off);
+  off += align256((size_t)BH * k * sizeof(int));
+  w.ccount = (int*)(base + off);
+  off += align256((size_t)BH * nchunk * k * sizeof(int));
+  w.cbase = (int*)(base + off);
+  off += align256((size_t)BH * nchunk * k * sizeof(int));
+  *total = off;
+  return w;
+}
+
+// centroid c of head bh = token floor(c*N/k), or the caller's warm start
+__global__ void km_init_kernel(const uint16_t* __restrict__ V, const float* __restrict__ init,
+                               float* __restrict__ cent, int N, int k) {
+  int bh = blockIdx.x, c = blockIdx.y, ch = threadIdx.x;
+  float* dst = cent + ((int64_t)bh * k + c) * 128;
+  if (init) {
+    dst[ch] = init[((int64_t)bh * k + c) * 128 + ch];
+  } else {
+    int64_t src = ((int64_t)c * N) / k;
+    dst[ch] = __uint_as_float((uint32_t)V[((int64_t)bh * N + src) * 128 + ch] << 16);
+  }
+}
+
+__global__ void __launch_bounds__(kAssignThreads) km_assign_kernel(const uint16_t* __restrict__ V,
+                                                                  const float* __restrict__ cent,
+                                                                  int32_t* __restrict__ assign,
+                                                                  int N, int k) {
+  extern __shared__ float4 cs4[];   // [k][32] float4 = [k][128] floats
+  const int bh = blockIdx.y;
+  const float4* src = reinterpret_cast<const float4*>(cent + (int64_t)bh * k * 128);
+  for (int i = threadIdx.x; i < k * 32; i += blockDim.x) cs4[i] = src[i];
+  __syncthreads();
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  uint32_t v[64];
+  const uint4* row = reinterpret_cast<const uint4*>(V + ((int64_t)bh * N + n) * 128);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    uint4 q = __ldg(row + i);
+    v[4 * i] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
+  }
+  int best = 0;
+  float bd = 0.0f;
+  for (int c = 0; c < k; ++c) {
+    const float4* cc = cs4 + c * 32;
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      float4 m = cc[i];
+      float x0 = __uint_as_float(v[2 * i] << 16), x1 = __uint_as_float(v[2 * i] & 0xFFFF0000u);
+      float x2 = __uint_as_float(v[2 * i + 1] << 16), x3 = __uint_as_float(v[2 * i + 1] & 0xFFFF0000u);
+      float t0 = __fsub_rn(x0, m.x), t1 = __fsub_rn(x1, m.y), t2 = __fsub_rn(x2, m.z), t3 = __fsub_rn(x3, m.w);
+      acc = __fmaf_rn(t0, t0, acc);
+      acc = __fmaf_rn(t1, t1, acc);
+      acc = __fmaf_rn(t2, t2, acc);
+      acc = __fmaf_rn(t3, t3, acc);
+    }
+    if (c == 0 || acc < bd) {
+      bd = acc;
+      best = c;
+    }
+  }
+  assign[(int64_t)bh * N + n] = best;
+}
+
+// Exact fixed-point sums per (cluster, channel) for one chunk of tokens; one
+// thread per channel walks the chunk in order (no atomics in shared memory),
+// then the chunk's partial sums are added to the head's totals.
+__global__ void __launch_bounds__(128) km_accum_kernel(const uint16_t* __restrict__ V,
+                                                      const int32_t* __restrict__ assign,
+                                                      long long* __restrict__ sums,
+                                                      int* __restrict__ counts, int N, int k) {
+  extern __shared__ long long acc[];   // [k][128]
+  __shared__ int cnt[VCA_MAX_CLUSTERS];
+  const int bh = blockIdx.y, ch = threadIdx.x;
+  for (int c = 0; c < k; ++c) acc[c * 128 + ch] = 0;
+  if (ch < k) cnt[ch] = 0;
+  __syncthreads();
+  const int n0 = blockIdx.x * kAccumChunk, n1 = min(N, n0 + kAccumChunk);
+  const uint16_t* vb = V + (int64_t)bh * N * 128;
+  const int32_t* ab = assign + (int64_t)bh * N;
+  for (int n = n0; n < n1; ++n) {
+    int a = __ldg(ab + n);
+    float v = __uint_as_float((uint32_t)__ldg(vb + (int64_t)n * 128 + ch) << 16);
+    acc[a * 128 + ch] += __float2ll_rn(v * 16777216.0f);
+    if (ch == 0) cnt[a] += 1;
+  }
+  __syncthreads();
+  long long* dst = sums + (int64_t)bh * k * 128;
+  for (int c = 0; c < k; ++c) {
+    long long s = acc[c * 128 + ch];
+    if (s != 0) atomicAdd(reinterpret_cast<unsigned long long*>(dst + c * 128 + ch), (unsigned long long)s);
+  }
+  if (ch < k && cnt[ch] != 0) atomicAdd(counts + (int64_t)bh * k + ch, cnt[ch]);
+}
+
+__global__ void km_update_kernel(const long long* __restrict__ sums, const int* __restrict__ counts,
+                                 float* __restrict__ cent, int k) {
+  int bh = blockIdx.x, c = blockIdx.y, ch = threadIdx.x;
+  int n = counts[(int64_t)bh * k + c];
+  if (n == 0) return;   // empty cluster keeps its centroid
+  long long s = sums[((int64_t)bh * k + c) * 128 + ch];
+  double m = __ddiv_rn((double)s, (double)n * 16777216.0);
+  cent[((int64_t)bh * k + c) * 128 + ch] = __double2float_rn(m);
+}
+
+// ---- stable counting sort by cluster
+__global__ void sort_count_kernel(const int32_t* __restrict__ assign, int* __restrict__ ccount,
+                                  int N, int k, int nchunk) {
+  __shared__ int h[VCA_MAX_CLUSTERS];
+  const int bh = blockIdx.y, chunk = blockIdx.x;
+  if (threadIdx.x < k) h[threadIdx.x] = 0;
+  __syncthreads();
+  const int n0 = chunk * kSortChunk, n1 = min(N, n0 + kSortChunk);
+  for (int n = n0 + threadIdx.x; n < n1; n += blockDim.x) atomicAdd(&h[assign[(int64_t)bh * N + n]], 1);
+  __syncthreads();
+  if (threadIdx.x < k) ccount[((int64_t)bh * nchunk + chunk) * k + threadIdx.x] = h[threadIdx.x];
+}
+
+// One CTA per head: base(chunk, c) = sum of all tokens of clusters < c plus the
+// tokens of cluster c in earlier chunks.
+__global__ void sort_scan_kernel(const int* __restrict__ ccount, int* __restrict__ cbase, int k,
+                                 int nchunk) {
+  __shared__ int tot[VCA_MAX_CLUSTERS];
+  __shared__ int off[VCA_MAX_CLUSTERS];
+  const int bh = blockIdx.x, c = threadIdx.x;
+  const int* cc = ccount + (int64_t)bh * nchunk * k;
+  int* cb = cbase + (int64_t)bh * nchunk * k;
+  if (c < k) {
+    int s = 0;
+    for (int j = 0; j < nchunk; ++j) s += cc[j * k + c];
+    tot[c] = s;
+  }
+  __syncthreads();
+  if (c == 0) {
+    int run = 0;
+    for (int i = 0; i < k; ++i) {
+      off[i] = run;
+      run += tot[i];
+    }
+  }
+  __syncthreads();
+  if (c < k) {
+    int run = off[c];
+    for (int j = 0; j < nchunk; ++j) {
+      cb[j * k + c] = run;
+      run += cc[j * k + c];
+    }
+  }
+}
+
+// One warp per chunk: tokens in index order, ranked inside each group of 32
+// by matching cluster ids, so equal clusters keep their original order.
+__global__ void __launch_bounds__(32) sort_scatter_kernel(const int32_t* __restrict__ assign,
+                                                         const int* __restrict__ cbase,
+                                                         int32_t* __restrict__ perm, int N, int k,
+                                                         int nchunk) {
+  __shared__ int base[VCA_MAX_CLUSTERS];
+  const int bh = blockIdx.y, chunk = blockIdx.x, lane = threadIdx.x;
+  for (int c = lane; c < k; c += 32) base[c] = cbase[((int64_t)bh * nchunk + chunk) * k + c];
+  __syncwarp();
+  const int n0 = chunk * kSortChunk, n1 = min(N, n0 + kSortChunk);
+  const int32_t* ab = assign + (int64_t)bh * N;
+  int32_t* pb = perm + (int64_t)bh * N;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int g = n0; g < n1; g += 32) {
+    int n = g + lane;
+    bool valid = n < n1;
+    unsigned active = __ballot_sync(0xffffffffu, valid);
+    int a = valid ? ab[n] : -1 - lane;     // invalid lanes never match a cluster
+    unsigned peers = __match_any_sync(0xffffffffu, a);
+    int pos = 0;
+    if (valid) pos = base[a] + __popc(peers & lt);
+    __syncwarp();
+    if (valid) {
+      pb[pos] = n;
+      if ((peers & lt) == 0) base[a] += __popc(peers & active);
+    }
+    __syncwarp();
+  }
+}
+
+}  // namespace vca
+
+using namespace vca;
+
+extern "C" size_t vca_cluster_permute_workspace_size(int B, int H, int N, int k) {
+  if (B < 1 || H < 1 || N < 1 || k < 1) return 0;
+  size_t total;
+  carve(nullptr, B * H, N, k, &total);
+  return total;
+}
+
+static int cluster_permute_impl(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
+                                const float* init, float* cent, int32_t* assign, int32_t* perm,
+                                const KmWs& w, cudaStream_t s) {
+  const int BH = B * H;
+  size_t sums_bytes = (size_t)BH * k * 128 * sizeof(long long);
+  size_t counts_bytes = (size_t)BH * k * sizeof(int);
+  km_init_kernel<<<dim3(BH, k), 128, 0, s>>>(V, init, cent, N, k);
+  int rc = check_launch("km_init_kernel");
+  if (rc) return rc;
+  const size_t assign_smem = (size_t)k * 128 * sizeof(float);
+  const size_t accum_smem = (size_t)k * 128 * sizeof(long long);
+  if (cudaFuncSetAttribute(km_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)assign_smem) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(km_accum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)accum_smem) !=
+          cudaSuccess)
+    return fail(VCA_ERR_CUDA, "vca_cluster_permute: cannot set shared-memory size");
+  const dim3 g_assign((N + kAssignThreads - 1) / kAssignThreads, BH);
+  const dim3 g_accum((N + kAccumChunk - 1) / kAccumChunk, BH);
+  for (int it = 0; it < iters; ++it) {
+    km_assign_kernel<<<g_assign, kAssignThreads, assign_smem, s>>>(V, cent, assign, N, k);
+    if ((rc = check_launch("km_assign_kernel"))) return rc;
+    if (cudaMemsetAsync(w.sums, 0, sums_bytes, s) != cudaSuccess ||
+        cudaMemsetAsync(w.counts, 0, counts_bytes, s) != cudaSuccess)
+      return fail(VCA_ERR_CUDA, "vca_cluster_permute: memset failed");
+    km_accum_kernel<<<g_accum, 128, accum_smem, s>>>(V, assign, w.sums, w.counts, N, k);
+    if ((rc = check_launch("km_accum_kernel"))) return rc;
+    km_update_kernel<<<dim3(BH, k), 128, 0, s>>>(w.sums, w.counts, cent, k);
+    if ((rc = check_launch("km_update_kernel"))) return rc;
+  }
+  const int nchunk = (N + kSortChunk - 1) / kSortChunk;
+  sort_count_kernel<<<dim3(nchunk, BH), 256, 0, s>>>(assign, w.ccount, N, k, nchunk);
+  if ((rc = check_launch("sort_count_kernel"))) return rc;
+  sort_scan_kernel<<<BH, 64, 0, s>>>(w.ccount, w.cbase, k, nchunk);
+  if ((rc = check_launch("sort_scan_kernel"))) return rc;
+  sort_scatter_kernel<<<dim3(nchunk, BH), 32, 0, s>>>(assign, w.cbase, perm, N, k, nchunk);
+  return check_launch("sort_scatter_kernel");
+}
+
+static int check_cluster_args(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
+                              const float* init, float* cent, int32_t* assign, int32_t* perm) {
+  if (d != VCA_HEAD_DIM) return fail(VCA_ERR_UNSUPPORTED, "vca_cluster_permute: d must be 128");
+  if (k < 1 || k > VCA_MAX_CLUSTERS)
+    return fail(VCA_ERR_UNSUPPORTED, "vca_cluster_permute: k must be in [1, %d]", VCA_MAX_CLUSTERS);
+  if (iters < 1 || iters > 64) return fail(VCA_ERR_INVALID, "vca_cluster_permute: iters must be in [1, 64]");
+  if (B < 1 || H < 1 || N < 1 || (int64_t)B * H > 65535 || N > (1 << 24))
+    return fail(VCA_ERR_INVALID, "vca_cluster_permute: bad shape B=%d H=%d N=%d", B, H, N);
+  if (!V || !cent || !assign || !perm) return fail(VCA_ERR_INVALID, "vca_cluster_permute: null pointer");
+  if (!aligned16(V) || !aligned16(cent) || (init && !aligned16(init)) || !aligned16(assign) || !aligned16(perm))
+    return fail(VCA_ERR_INVALID, "vca_cluster_permute: pointers must be 16-byte aligned");
+  return VCA_OK;
+}
+
+extern "C" int vca_cluster_permute(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
+                                   const float* init_centroids, float* centroids, int32_t* assign,
+                                   int32_t* perm, void* ws, size_t ws_bytes, vca_stream_t stream) {
+  int rc = check_cluster_args(V, B, H, N, d, k, iters, init_centroids, centroids, assign, perm);
+  if (rc) return rc;
+  size_t need = vca_cluster_permute_workspace_size(B, H, N, k);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(VCA_ERR_WORKSPACE, "vca_cluster_permute: workspace needs %zu bytes", need);
+  size_t total;
+  KmWs w = carve(ws, B * H, N, k, &total);
+  return cluster_permute_impl(V, B, H, N, d, k, iters, init_centroids, centroids, assign, perm, w,
+                              (cudaStream_t)stream);
+}

@@ -1,0 +1,230 @@
+"""Thin ctypes binding of libvca.so (argument marshalling only).
+
+Every computation runs in the library's CUDA kernels; this module allocates the
+caller-owned device buffers with PyTorch, passes their pointers and the current
+CUDA stream, and turns non-zero status codes into exceptions.  It fails loudly
+when the library has not been built: there is no CPU fallback.
+
+Names follow the C ABI in include/vca.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libvca.so")
+HEAD_DIM = 128
+BLOCK = 128
+
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_NONFINITE, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5, -6
+_NAMES = {0: "VCA_OK", -1: "VCA_ERR_INVALID", -2: "VCA_ERR_UNSUPPORTED", -3: "VCA_ERR_CUDA",
+          -4: "VCA_ERR_TIMEOUT", -5: "VCA_ERR_NONFINITE", -6: "VCA_ERR_WORKSPACE"}
+
+_lib = None
+
+EXPORTED = [
+    "vca_status_bytes", "vca_reset_status", "vca_check_status", "vca_last_error",
+    "vca_set_wait_limit_ns", "vca_debug_wait_timeout", "vca_expcast_ref", "vca_e4m3_encode",
+    "vca_cluster_permute_workspace_size", "vca_cluster_permute",
+    "vca_smooth_quantize_workspace_size", "vca_smooth_quantize_qkv",
+    "vca_attention_workspace_size", "vca_attention_fwd",
+    "vca_bf16_attention_workspace_size", "vca_bf16_attention_fwd",
+]
+
+
+class VcaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built; run `python -m bit_attention_video_02_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+        L.vca_status_bytes.restype = sz
+        L.vca_reset_status.argtypes = [vp, vp]
+        L.vca_check_status.argtypes = [vp, vp, ctypes.POINTER(i32), ctypes.POINTER(i32)]
+        L.vca_last_error.restype = ctypes.c_char_p
+        L.vca_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.vca_debug_wait_timeout.argtypes = [vp, ctypes.c_uint64, vp]
+        L.vca_expcast_ref.argtypes = [vp, vp, i64, vp]
+        L.vca_e4m3_encode.argtypes = [vp, vp, i64, vp]
+        L.vca_cluster_permute_workspace_size.restype = sz
+        L.vca_cluster_permute_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.vca_cluster_permute.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.vca_smooth_quantize_workspace_size.restype = sz
+        L.vca_smooth_quantize_workspace_size.argtypes = [i32, i32, i32]
+        L.vca_smooth_quantize_qkv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32] + [vp] * 7 + [vp, sz, vp]
+        L.vca_attention_workspace_size.restype = sz
+        L.vca_attention_workspace_size.argtypes = [i32, i32, i32]
+        L.vca_attention_fwd.argtypes = [vp] * 7 + [i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+        L.vca_bf16_attention_workspace_size.restype = sz
+        L.vca_bf16_attention_workspace_size.argtypes = [i32, i32, i32]
+        L.vca_bf16_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+        for fn in ("vca_reset_status", "vca_check_status", "vca_debug_wait_timeout", "vca_expcast_ref",
+                   "vca_e4m3_encode", "vca_cluster_permute", "vca_smooth_quantize_qkv",
+                   "vca_attention_fwd", "vca_bf16_attention_fwd"):
+            getattr(L, fn).restype = i32
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise VcaError(rc, lib().vca_last_error().decode(errors="replace"))
+
+
+class Workspace:
+    """Caller-owned device scratch; its first bytes hold the device status word."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        self.nbytes = max(int(nbytes), 256)
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+
+    def ensure(self, nbytes: int):
+        if nbytes > self.nbytes:
+            self.__init__(nbytes, self.buf.device)
+        return self
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+    def check(self, stream=None):
+        where, info = ctypes.c_int(0), ctypes.c_int(0)
+        rc = lib().vca_check_status(self.ptr, _stream(stream), ctypes.byref(where), ctypes.byref(info))
+        if rc != OK:
+            raise VcaError(rc, lib().vca_last_error().decode(errors="replace"))
+
+
+def set_wait_limit_ns(ns: int):
+    lib().vca_set_wait_limit_ns(int(ns))
+
+
+def debug_wait_timeout(ws: Workspace, limit_ns: int, stream=None):
+    _check(lib().vca_debug_wait_timeout(ws.ptr, int(limit_ns), _stream(stream)))
+
+
+# ------------------------------------------------------------------ ExpCast / E4M3
+def expcast_ref(z: torch.Tensor, stream=None) -> torch.Tensor:
+    assert z.is_cuda and z.dtype == torch.float32 and z.is_contiguous()
+    out = torch.empty(z.shape, dtype=torch.uint8, device=z.device)
+    _check(lib().vca_expcast_ref(_ptr(z), _ptr(out), z.numel(), _stream(stream)))
+    return out
+
+
+def e4m3_encode(x: torch.Tensor, stream=None) -> torch.Tensor:
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(lib().vca_e4m3_encode(_ptr(x), _ptr(out), x.numel(), _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ V-Smooth
+def _bhnd(x):
+    assert x.is_cuda and x.dtype == torch.bfloat16 and x.is_contiguous() and x.dim() == 4, \
+        "expected contiguous bf16 CUDA tensor [B, H, N, d]"
+    return x.shape
+
+
+def cluster_permute(V: torch.Tensor, k: int, iters: int = 3, init=None, ws: Workspace | None = None,
+                    stream=None):
+    B, H, N, d = _bhnd(V)
+    dev = V.device
+    cent = torch.empty(B, H, k, d, dtype=torch.float32, device=dev)
+    assign = torch.empty(B, H, N, dtype=torch.int32, device=dev)
+    perm = torch.empty(B, H, N, dtype=torch.int32, device=dev)
+    need = lib().vca_cluster_permute_workspace_size(B, H, N, k)
+    ws = (ws or Workspace(need, dev)).ensure(need)
+    if init is not None:
+        assert init.shape == (B, H, k, d) and init.dtype == torch.float32 and init.is_contiguous()
+    _check(lib().vca_cluster_permute(_ptr(V), B, H, N, d, k, iters, _ptr(init), _ptr(cent), _ptr(assign),
+                                     _ptr(perm), ws.ptr, ws.nbytes, _stream(stream)))
+    return cent, assign, perm
+
+
+def alloc_quantized(B, H, N, device="cuda"):
+    nb = (N + BLOCK - 1) // BLOCK
+    Np = nb * BLOCK
+    u8, f32 = torch.uint8, torch.float32
+    return dict(
+        Qq=torch.empty(B, H, Np, HEAD_DIM, dtype=u8, device=device),
+        q_scale=torch.empty(B, H, nb, dtype=f32, device=device),
+        Kq=torch.empty(B, H, Np, HEAD_DIM, dtype=u8, device=device),
+        k_scale=torch.empty(B, H, nb, dtype=f32, device=device),
+        VrT=torch.empty(B, H, HEAD_DIM, Np, dtype=u8, device=device),
+        v_exp=torch.empty(B, H, nb, dtype=torch.int8, device=device),
+        v_mean=torch.empty(B, H, nb, HEAD_DIM, dtype=torch.bfloat16, device=device))
+
+
+def smooth_quantize(Q, K, V, perm, out=None, ws: Workspace | None = None, stream=None):
+    B, H, N, d = _bhnd(Q)
+    assert K.shape == Q.shape and V.shape == Q.shape
+    assert perm.is_cuda and perm.dtype == torch.int32 and perm.shape == (B, H, N) and perm.is_contiguous()
+    o = out or alloc_quantized(B, H, N, Q.device)
+    need = lib().vca_smooth_quantize_workspace_size(B, H, N)
+    ws = (ws or Workspace(need, Q.device)).ensure(need)
+    _check(lib().vca_smooth_quantize_qkv(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), B, H, N, d, BLOCK, _ptr(o["Qq"]), _ptr(o["q_scale"]),
+        _ptr(o["Kq"]), _ptr(o["k_scale"]), _ptr(o["VrT"]), _ptr(o["v_exp"]), _ptr(o["v_mean"]),
+        ws.ptr, ws.nbytes, _stream(stream)))
+    return o
+
+
+# ------------------------------------------------------------------ attention
+def attention_fwd(ops: dict, N: int, softmax_scale: float | None = None, O=None, lse=None,
+                  want_lse: bool = False, ws: Workspace | None = None, stream=None):
+    B, H, Np, d = ops["Qq"].shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dev = ops["Qq"].device
+    if O is None:
+        O = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    need = lib().vca_attention_workspace_size(B, H, N)
+    ws = (ws or Workspace(need, dev)).ensure(need)
+    _check(lib().vca_attention_fwd(
+        _ptr(ops["Qq"]), _ptr(ops["q_scale"]), _ptr(ops["Kq"]), _ptr(ops["k_scale"]), _ptr(ops["VrT"]),
+        _ptr(ops["v_exp"]), _ptr(ops["v_mean"]), B, H, N, d, scale, _ptr(O), _ptr(lse), ws.ptr, ws.nbytes,
+        _stream(stream)))
+    return (O, lse) if want_lse else O
+
+
+def bf16_attention_fwd(Q, K, V, softmax_scale: float | None = None, O=None, lse=None, want_lse=False,
+                       ws: Workspace | None = None, stream=None):
+    B, H, N, d = _bhnd(Q)
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    if O is None:
+        O = torch.empty_like(Q)
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=Q.device)
+    need = lib().vca_bf16_attention_workspace_size(B, H, N)
+    ws = (ws or Workspace(need, Q.device)).ensure(need)
+    _check(lib().vca_bf16_attention_fwd(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, scale, _ptr(O), _ptr(lse),
+                                        ws.ptr, ws.nbytes, _stream(stream)))
+    return (O, lse) if want_lse else O
+
+
+def vc_attention(Q, K, V, k: int = 32, iters: int = 3, softmax_scale=None, perm=None, ws=None, stream=None):
+    """Whole path: cluster/permute (unless `perm` is given), quantise, attend."""
+    if perm is None:
+        _, _, perm = cluster_permute(V, k, iters, ws=ws, stream=stream)
+    ops = smooth_quantize(Q, K, V, perm, ws=ws, stream=stream)
+    return attention_fwd(ops, Q.shape[2], softmax_scale, ws=ws, stream=stream)

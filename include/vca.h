@@ -1,0 +1,190 @@
+/*
+ * vca.h -- C ABI of libvca.so: VC-Attention-style FP8 self-attention forward
+ * for video diffusion-transformer token sequences, on B200 (sm_100a).
+ *
+ * The method (no code is published; described on these pages):
+ *   [VCA-news] "VC-Attention: Training-Free Low-Bit Attention Speeds Video
+ *              Diffusion Up to 3.6x" (agihunt.info): V-Smooth bullet (reorder
+ *              value tokens by lightweight online clustering, quantise only the
+ *              residual after the block mean, restore the mean from the online
+ *              softmax row sums) and ExpCast-FP8 bullet (score -> E4M3
+ *              probability code with one fused multiply-add).
+ *   [VCA-mtp]  "Nunchux AI Introduces VC-Attention: A Training-Free Low-Bit
+ *              Attention Kernel That Speeds Up Video Diffusion Transformers"
+ *              (MarkTechPost abstract): byte ~ 8 log2(v) + 56, beta = -0.35,
+ *              0.125 bit per value element for the mean, block sorting.
+ *   [VCA-ru]   "VC-Attention" (aikraft.ru), section "Решение": k-means
+ *              grouping, mean stored exactly, one FMA per probability byte.
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are DEVICE pointers owned by the caller, contiguous,
+ *    16-byte aligned (VCA_ERR_INVALID otherwise).  The library allocates no
+ *    device memory; scratch space is the caller's workspace `ws` of at least
+ *    the size the matching *_workspace_size() returns.  The first 16 bytes of
+ *    every workspace are the device status word; zero the workspace once after
+ *    allocating it (vca_reset_status does this).
+ *  - bf16 tensors are passed as uint16_t bit patterns (vca_bf16).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default).
+ *    The return value reports argument and launch errors only; errors found on
+ *    the device (a bounded wait that ran out, non-finite input) are recorded
+ *    in the workspace status word and returned by vca_check_status().
+ *  - Layouts: B batch, H heads, N tokens, d = 128 head channels,
+ *    nb = ceil(N/128) blocks of 128 tokens, Np = 128*nb.  Q/K/V/O are
+ *    [B][H][N][d] row-major.
+ *  - Thread safety: calls are independent; two calls that share a workspace
+ *    must not run concurrently on the GPU.
+ */
+#ifndef VCA_H
+#define VCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t vca_bf16;
+typedef struct CUstream_st* vca_stream_t; /* same type as cudaStream_t */
+
+#define VCA_OK 0
+#define VCA_ERR_INVALID (-1)     /* null pointer, bad shape or alignment        */
+#define VCA_ERR_UNSUPPORTED (-2) /* d != 128, block != 128, k or N out of range */
+#define VCA_ERR_CUDA (-3)        /* a CUDA launch / runtime call failed         */
+#define VCA_ERR_TIMEOUT (-4)     /* a device-side bounded wait ran out          */
+#define VCA_ERR_NONFINITE (-5)   /* an input held inf/NaN (prep kernels)        */
+#define VCA_ERR_WORKSPACE (-6)   /* workspace missing or smaller than required  */
+
+#define VCA_HEAD_DIM 128
+#define VCA_BLOCK 128
+#define VCA_MAX_CLUSTERS 64
+
+/* ------------------------------------------------------------------ status */
+
+/* Bytes of the status word at the start of every workspace. */
+size_t vca_status_bytes(void);
+
+/* Zeroes the status word of `ws` (asynchronously on `stream`). */
+int vca_reset_status(void* ws, vca_stream_t stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded in `ws`
+ * since the last reset (VCA_OK if none) and clears it.  If `where`/`info` are
+ * non-null they receive the kernel's location tag and detail. */
+int vca_check_status(void* ws, vca_stream_t stream, int* where, int* info);
+
+/* Message for the most recent failing call made by this host thread. */
+const char* vca_last_error(void);
+
+/* Device-side wait limit in nanoseconds for every bounded wait (default
+ * 2e9).  Process-wide; takes effect for launches made after the call. */
+void vca_set_wait_limit_ns(uint64_t ns);
+
+/* Self-test of the bounded-wait path: launches one block that waits on an
+ * mbarrier no thread ever arrives on, with a limit of `limit_ns`; the wait
+ * runs out and VCA_ERR_TIMEOUT is recorded in `ws` (read it with
+ * vca_check_status).  It faults nothing and returns in ~limit_ns. */
+int vca_debug_wait_timeout(void* ws, uint64_t limit_ns, vca_stream_t stream);
+
+/* ------------------------------------------------------------------ ExpCast */
+
+/* ExpCast-FP8 reference map ([VCA-news] ExpCast-FP8 bullet; [VCA-mtp]: an
+ * E4M3 byte read as an integer is ~8 log2(v) + 56, beta = -0.35).
+ * For each of the n fp32 log2-domain, max-subtracted scores z[i]:
+ *   codes[i] = clamp(rne(fmaf(8, z[i], 55.65f)), 0, 126)   (E4M3 byte of ~2^z)
+ * with z = -inf -> 0 and z = NaN -> 0x7F.  z: n floats; codes: n bytes. */
+int vca_expcast_ref(const float* z, uint8_t* codes, int64_t n, vca_stream_t stream);
+
+/* E4M3 encoder used by the prep kernels: out[i] = e4m3(x[i]), round to nearest
+ * even, finite values saturated to +-448 (hardware cvt ... satfinite).
+ * x: n floats; out: n bytes. */
+int vca_e4m3_encode(const float* x, uint8_t* out, int64_t n, vca_stream_t stream);
+
+/* ------------------------------------------------------------------ V-Smooth */
+
+size_t vca_cluster_permute_workspace_size(int B, int H, int N, int k);
+
+/* V-Smooth grouping ([VCA-news]: value tokens reordered by lightweight online
+ * clustering; [VCA-ru] "Решение": k-means groups similar tokens into blocks;
+ * [VCA-mtp]: block means remove most energy after sorting).
+ * Per (b, h) independently, Lloyd k-means on the value vectors:
+ *   init: centroid c = V[floor(c*N/k)], or init_centroids [B][H][k][d] if
+ *         non-null (warm start, e.g. from an earlier denoising step);
+ *   iters rounds of: assign each token to the nearest centroid (fp32 squared
+ *   distance accumulated with one fma per channel in channel order, ties to the
+ *   lowest index), then centroid = exact mean of its members (2^-24 fixed-point
+ *   sum, one fp64 division; an empty cluster keeps its centroid).
+ * Then a stable counting sort by cluster gives perm[new] = old index.
+ *   V          [B][H][N][d] bf16        (in)
+ *   centroids  [B][H][k][d] fp32        (out)
+ *   assign     [B][H][N] int32          (out, the assignment of the last round)
+ *   perm       [B][H][N] int32          (out)
+ * 1 <= k <= VCA_MAX_CLUSTERS, 1 <= iters <= 64, |V| < 2^20. */
+int vca_cluster_permute(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
+                        const float* init_centroids, float* centroids, int32_t* assign,
+                        int32_t* perm, void* ws, size_t ws_bytes, vca_stream_t stream);
+
+size_t vca_smooth_quantize_workspace_size(int B, int H, int N);
+
+/* V-Smooth quantisation ([VCA-news] V-Smooth bullet; [VCA-ru] "Решение": the
+ * block mean is subtracted and stored exactly, only the residual is quantised;
+ * [VCA-mtp]: 0.125 bit per value element for the mean).
+ * Per (b, h) and block of 128 permuted tokens (the tail block holds N mod 128):
+ *   K and V rows are gathered by perm; Q keeps the original order.
+ *   v_mean[b][c]  = bf16(exact mean of V over the block's tokens)
+ *   residual r    = V - v_mean (fp32);  v_exp[b] = smallest e with
+ *                   max|r| <= 448 * 2^e (0 if r == 0), clamped to [-127, 127]
+ *   VrT[c][j]     = e4m3(r * 2^-e)   (transposed: channel-major, Np tokens)
+ *   Q/K blocks:   scale = max|x| / 448 (fp32), codes = e4m3(x * (448/max|x|))
+ *                 (an all-zero block: scale 1, codes 0)
+ *   e4m3() rounds to nearest even and saturates at +-448; padding (N..Np) is 0.
+ * Outputs (all device):
+ *   Qq [B][H][Np][d] u8, q_scale [B][H][nb] f32, Kq [B][H][Np][d] u8 (permuted),
+ *   k_scale [B][H][nb] f32, VrT [B][H][d][Np] u8 (permuted), v_exp [B][H][nb] i8,
+ *   v_mean [B][H][nb][d] bf16.
+ * block must be 128.  Non-finite or |x| >= 2^20 inputs record
+ * VCA_ERR_NONFINITE in the status word. */
+int vca_smooth_quantize_qkv(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V,
+                            const int32_t* perm, int B, int H, int N, int d, int block,
+                            uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                            uint8_t* VrT, int8_t* v_exp, vca_bf16* v_mean, void* ws,
+                            size_t ws_bytes, vca_stream_t stream);
+
+/* ------------------------------------------------------------------ attention */
+
+size_t vca_attention_workspace_size(int B, int H, int N);
+
+/* ExpCast-FP8 attention forward, non-causal self-attention ([VCA-news]:
+ * low-bit QK^T and PV, ExpCast-FP8 softmax, mean restored from the row sums
+ * online softmax keeps).  For each query row i (original order) of head (b,h),
+ * visiting the key blocks b = 0..nb-1 in (permuted) order:
+ *   z_ij  = (Qq_i . Kq_j) * q_scale * k_scale * softmax_scale * log2(e)
+ *   n_b   = ceil(max_{j in b} z_ij - phi), phi = 0.65/8 (block max on the grid)
+ *   n     = reference: n_0 at the first block; it moves up to n_b only when
+ *           n_b > n + 4, and everything accumulated so far is then scaled by
+ *           the exact power of two 2^(n_old - n_b)
+ *   p_ij  = E4M3 value of clamp(rne(8 z_ij + 55 + 32 - 8 n), 0, 126)
+ *           (ExpCast-FP8 of the probability relative to n + phi, pre-scaled by
+ *           2^4; every code stays <= 120)
+ *   l_ib  = sum of p_ij over key block b
+ *   O_i   = (sum_b 2^v_exp[b] sum_{j in b} p_ij VrT[:, j] + sum_b l_ib v_mean[b])
+ *           / sum_b l_ib          -> O [B][H][N][d] bf16 (round to nearest even)
+ *   lse_i = ln 2 * (n + phi - 4 + log2 sum_b l_ib)    (optional, [B][H][N] fp32)
+ * Inputs are the outputs of vca_smooth_quantize_qkv; |z| must stay below 2^18.
+ * The workspace needs only the status word (vca_attention_workspace_size). */
+int vca_attention_fwd(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                      const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                      const vca_bf16* v_mean, int B, int H, int N, int d, float softmax_scale,
+                      vca_bf16* O, float* lse, void* ws, size_t ws_bytes, vca_stream_t stream);
+
+/* In-repo BF16 comparator: exact-softmax flash attention (online softmax with
+ * exp2), tcgen05 BF16 MMAs with fp32 accumulation in tensor memory.
+ *   Q, K, V, O [B][H][N][d] bf16; lse [B][H][N] fp32 natural log (nullable). */
+size_t vca_bf16_attention_workspace_size(int B, int H, int N);
+int vca_bf16_attention_fwd(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V, int B, int H,
+                           int N, int d, float softmax_scale, vca_bf16* O, float* lse, void* ws,
+                           size_t ws_bytes, vca_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VCA_H */

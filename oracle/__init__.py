@@ -31,6 +31,7 @@ IDENTITY_QUANT = 2
 PLANT_TRUNC = 64
 PLANT_NO_MEAN = 128
 PLANT_BETA0 = 256
+PLANT_NO_RESCALE = 512
 BLOCK = 128
 
 _lib = None

@@ -331,41 +331,61 @@ void vo_smooth_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_
  * multiple of 8 (an exact power-of-two rescale). */
 #define VO_PHI (0.65 / 8.0)
 
-/* READING: probabilities are encoded relative to a reference 4 octaves below
- * the snapped row maximum, i.e. the byte written is ExpCast of z - m + 4: the
- * row maximum lands on codes 80..88 (p between 8 and 16) instead of 48..56.
- * This fixed power-of-two pre-scale cancels in the normalisation; it moves the
- * E4M3 underflow tail 4 octaves further from the maximum and leaves 4 octaves
- * (codes up to 120 < 126) for a running maximum that lags the true one. */
+/* READING: probabilities are encoded 4 octaves above the reference, i.e. the
+ * byte written is ExpCast of z - m + 4: a maximum equal to the reference lands
+ * on codes 80..88 (p between 8 and 16) instead of 48..56.  This fixed
+ * power-of-two pre-scale cancels in the normalisation; it moves the E4M3
+ * underflow tail 4 octaves further from the maximum.  The reference may lag
+ * the running maximum by up to VO_LAG = 4 octaves (codes up to 120 < 126). */
 #define VO_HEADROOM 4
+#define VO_LAG 4
 
 /* One query row of the same-algorithm attention ([VCA-news] V-Smooth and
  * ExpCast-FP8 bullets: the block mean is restored from the row sums that
  * online softmax keeps).  Operands are decoded values in fp64:
  *   q[d] and its block scale qs; kh[N][d], ks[N] (permuted keys and their
  *   block scales); rh[N][d] residual codes decoded; vexp[nb]; mu[nb][d].
- * Steps: s_j = q.k_j; z_j = s_j*qs*ks_j*scale*log2(e); m = snapped max;
- * p_j = decode(ExpCast code of z_j - m); l_b = sum of p_j over block b;
- * acc = sum_b 2^vexp_b * sum_{j in b} p_j r_j + sum_b l_b mu_b;
- * O = acc / sum_b l_b. */
+ * Key blocks are visited in order, as online softmax does:
+ *   s_j = q.k_j;  z_j = s_j*qs*ks_j*scale*log2(e)
+ *   n_b = ceil(max_{j in b} z_j - phi)      (block maximum on the phi grid)
+ *   the reference n is set by the first block and moves up to n_b only when
+ *   n_b > n + VO_LAG; the accumulators are then scaled by 2^(n_old - n_b)
+ *   p_j = decode(clamp(rne(8 z_j + 55 + 8*VO_HEADROOM - 8 n), 0, 126))
+ *   l_b = sum_{j in b} p_j
+ *   acc += 2^vexp_b sum_{j in b} p_j r_j + l_b mu_b;  L += l_b
+ *   O = acc / L.
+ * READING: the pages name online softmax but not its rescale rule; this one
+ * (a reference that lags the running maximum by at most VO_LAG octaves) keeps
+ * every code <= 56 + 8*(VO_HEADROOM + VO_LAG) = 120 < 126. */
 static void attn_row(const double* q, double qs, const double* kh, const double* ks,
                      const double* rh, const int* vexp, const double* mu, int N, int d,
                      double softmax_scale, int flags, double* O, double* lse,
                      double* lblk, double* z /* scratch [N] */, double* acc /* [d] */) {
     const double log2e = 1.4426950408889634074;
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
-    double zmax = -INFINITY;
     for (int j = 0; j < N; ++j) {
         double s = 0.0;
         for (int c = 0; c < d; ++c) s += q[c] * kh[(int64_t)j * d + c];
         z[j] = s * qs * ks[j] * softmax_scale * log2e;
-        if (z[j] > zmax) zmax = z[j];
     }
-    double n = ceil(zmax - VO_PHI);
     for (int c = 0; c < d; ++c) acc[c] = 0.0;
-    double ltot = 0.0;
+    double ltot = 0.0, n = 0.0;
     for (int b = 0; b < nb; ++b) {
         int j0 = b * VO_BLOCK, j1 = j0 + VO_BLOCK < N ? j0 + VO_BLOCK : N;
+        double zmax = -INFINITY;
+        for (int j = j0; j < j1; ++j)
+            if (z[j] > zmax) zmax = z[j];
+        double nblk = ceil(zmax - VO_PHI);
+        if (b == 0) {
+            n = nblk;
+        } else if (nblk > n + VO_LAG) {
+            double sc = (flags & VO_PLANT_NO_RESCALE) ? 1.0 : exp2(n - nblk);   /* exact power of two */
+            for (int c = 0; c < d; ++c) acc[c] *= sc;
+            ltot *= sc;
+            if (lblk)
+                for (int b2 = 0; b2 < b; ++b2) lblk[b2] *= sc;
+            n = nblk;
+        }
         double lb = 0.0;
         double pv[512];
         for (int c = 0; c < d; ++c) pv[c] = 0.0;
@@ -374,7 +394,7 @@ static void attn_row(const double* q, double qs, const double* kh, const double*
             if (flags & VO_EXACT_EXP) {
                 p = exp2(z[j] - (n + VO_PHI) + VO_HEADROOM);
             } else {
-                /* = 8(z - m) + 55.65 + 8*VO_HEADROOM, m = n + phi */
+                /* = 8(z - m) + 55.65 + 8*VO_HEADROOM with m = n + phi */
                 double x = 8.0 * z[j] + 55.0 - 8.0 * n + 8.0 * VO_HEADROOM;
                 if (flags & VO_PLANT_BETA0) x += 0.35;
                 double r = (flags & VO_PLANT_TRUNC) ? floor(x) : nearbyint(x);

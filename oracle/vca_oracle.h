@@ -38,6 +38,7 @@ extern "C" {
 #define VO_PLANT_TRUNC     64  /* planted mistake: ExpCast truncates instead of RNE  */
 #define VO_PLANT_NO_MEAN   128 /* planted mistake: drop the rowsum*mean restore term */
 #define VO_PLANT_BETA0     256 /* planted mistake: addend 56 instead of 56 + beta    */
+#define VO_PLANT_NO_RESCALE 512 /* planted mistake: reference moves without rescaling */
 
 /* E4M3 (OCP FP8: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
  * no infinities, NaN = S.1111.111, largest finite 448). */

@@ -1,0 +1,67 @@
+"""CPU checks of the C-ABI library: it loads and exports every declared symbol;
+argument validation runs on the host and needs no GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_attention_video_02_b200 import build, vca
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "vca.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(vca_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return vca.lib()
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 16
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    assert sorted(vca.EXPORTED) == sorted(n for n in names if n in vca.EXPORTED)
+
+
+def test_workspace_queries(L):
+    assert L.vca_status_bytes() == 16
+    assert L.vca_smooth_quantize_workspace_size(1, 2, 1024) >= 16
+    small = L.vca_cluster_permute_workspace_size(1, 2, 1024, 8)
+    big = L.vca_cluster_permute_workspace_size(1, 40, 75600, 32)
+    assert small >= 16 and big > small
+    assert L.vca_cluster_permute_workspace_size(0, 1, 1, 1) == 0
+
+
+def test_host_argument_validation_needs_no_gpu(L):
+    # d != 128 and bad k are rejected before anything touches the device
+    rc = L.vca_cluster_permute(None, 1, 1, 16, 64, 4, 3, None, None, None, None, None, 0, None)
+    assert rc == vca.ERR_UNSUPPORTED
+    rc = L.vca_cluster_permute(None, 1, 1, 16, 128, 0, 3, None, None, None, None, None, 0, None)
+    assert rc == vca.ERR_UNSUPPORTED
+    rc = L.vca_smooth_quantize_qkv(None, None, None, None, 1, 1, 16, 128, 64, *([None] * 7), None, 0, None)
+    assert rc == vca.ERR_UNSUPPORTED
+    rc = L.vca_attention_fwd(*([None] * 7), 1, 1, 16, 128, 0.1, None, None, None, 0, None)
+    assert rc == vca.ERR_INVALID
+    rc = L.vca_expcast_ref(None, None, -1, None)
+    assert rc == vca.ERR_INVALID
+    assert b"n < 0" in L.vca_last_error()
+    rc = L.vca_bf16_attention_fwd(None, None, None, 1, 1, 16, 96, 0.1, None, None, None, 0, None)
+    assert rc == vca.ERR_UNSUPPORTED
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "bit_attention_video_02_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "vca_oracle" not in txt and "liboracle" not in txt, f

@@ -390,6 +390,30 @@ def test_same_algorithm_reduces_to_exact(N):
     assert np.abs(bad - exact).max() > 1e-3
 
 
+def test_online_rescale_reduces_to_exact():
+    # later key blocks score much higher, so the running reference moves up by
+    # more than 4 octaves several times; with exact exponentials and identity
+    # quantisers the online result must still equal exact attention
+    rng = np.random.default_rng(21)
+    N = 900
+    kf = rng.standard_normal((N, 128))
+    kf *= (1.0 + np.arange(N) // 128)[:, None] * 1.5
+    qf = np.abs(rng.standard_normal((N, 128))) * 0.5
+    Q, K, V = bf16_bits_of(qf), bf16_bits_of(np.abs(kf)), _bits(rng, N)
+    perm = np.arange(N, dtype=np.int32)
+    sc = 1 / math.sqrt(128)
+    exact = oracle.exact_attention_head(Q, K, V, sc)
+    fl = oracle.EXACT_EXP | oracle.IDENTITY_QUANT
+    red = oracle.attention_head_bf16(Q, K, V, perm, sc, flags=fl)
+    assert np.abs(red - exact).max() < 1e-12
+    bad = oracle.attention_head_bf16(Q, K, V, perm, sc, flags=fl | oracle.PLANT_NO_RESCALE)
+    assert np.abs(bad - exact).max() > 1e-2
+    # with ExpCast codes the largest code stays <= 120 (never the 126 clamp)
+    ops = oracle.smooth_quantize_head(Q, K, V, perm)
+    O, _, lblk = oracle.attention_head(ops, N, sc, rows=np.arange(0, N, 50, dtype=np.int32), want_lblk=True)
+    assert np.all(np.isfinite(O)) and np.all(lblk <= 128 * 256.0)
+
+
 @pytest.mark.parametrize("N", [200, 1000])
 def test_same_algorithm_fidelity_and_row_sums(N):
     rng = np.random.default_rng(13)
