@@ -1,0 +1,389 @@
+"""Benchmark: V-Smooth prep + ExpCast-FP8 attention on one B200 per rank.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 3] [--no-cpu-baseline] [--no-e2e]
+
+One step is one pass of the whole hot path over one synthetic layer input:
+k-means over V + stable permutation (vca_cluster_permute), V-Smooth
+quantisation of Q/K/V (vca_smooth_quantize_qkv) and ExpCast-FP8 attention
+(vca_attention_fwd).  `value` is 4*B*H*N^2*d / (step time), i.e. attention
+TFLOP/s counting the prep inside the step, summed over ranks (each rank runs
+its own layer: weak scaling, no collective on the data path).
+
+Rank 0 prints one JSON line.  Multi-GPU runs are launched with
+torch.distributed.run (one rank per GPU); the timed region is bracketed by a
+barrier and synchronize, and the time is the max over ranks.
+
+--impl reference times the plain CPU oracle on the host cores (the method has
+no other reference implementation) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_attention_video_02_b200 import build as vca_build  # noqa: E402
+from bit_attention_video_02_b200 import vca  # noqa: E402
+from bit_attention_video_02_b200 import workloads as W  # noqa: E402
+
+METRIC = "FP8 attention TFLOP/s (4*B*H*N^2*d/t) & % of B200 FP8 peak; V-Smooth prep ms"
+KMEANS_ITERS = 3
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_PER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio (4.5 / 2.25 PFLOP/s)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, world, rank, local):
+    vca_build.build()
+    w = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local)
+    scale = 1.0 / math.sqrt(w.d)
+    Q, K, V = W.make_qkv(w, dev)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    ws = vca.Workspace(vca.lib().vca_cluster_permute_workspace_size(B, H, N, w.k), dev)
+    ops = vca.alloc_quantized(B, H, N, dev)
+    O = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 1 + 3 * KMEANS_ITERS + 3 + 1 + 1   # init, (assign, accum, update) x T, sort x3, quant, attn
+
+    def step(t_attn=None):
+        _, _, perm = vca.cluster_permute(V, w.k, KMEANS_ITERS, ws=ws)
+        vca.smooth_quantize(Q, K, V, perm, out=ops, ws=ws)
+        if t_attn is not None:
+            t_attn[0].record(stream)
+        vca.attention_fwd(ops, N, scale, O=O, ws=ws)
+        if t_attn is not None:
+            t_attn[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ws.check()
+
+    # ---- timed: whole step, device resident inputs (inputs exceed L2: no flush needed)
+    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for i in range(args.steps):
+            step(ev_a[i])
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ws.check()
+    t_total = e0.elapsed_time(e1) / 1e3
+    t_attn = statistics.mean(a.elapsed_time(b) for a, b in ev_a) / 1e3
+    t_total = max_over_ranks(t_total, world)
+    t_attn = max_over_ranks(t_attn, world)
+
+    # ---- prep alone (cluster + quantise) and the reuse path (quantise only)
+    _, _, perm = vca.cluster_permute(V, w.k, KMEANS_ITERS, ws=ws)
+    reps = max(3, args.steps)
+    p0, p1, q1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    torch.cuda.synchronize()
+    p0.record(stream)
+    for _ in range(reps):
+        _, _, perm = vca.cluster_permute(V, w.k, KMEANS_ITERS, ws=ws)
+        vca.smooth_quantize(Q, K, V, perm, out=ops, ws=ws)
+    p1.record(stream)
+    for _ in range(reps):
+        vca.smooth_quantize(Q, K, V, perm, out=ops, ws=ws)
+    q1.record(stream)
+    torch.cuda.synchronize()
+    prep_ms = p0.elapsed_time(p1) / reps
+    quant_ms = p1.elapsed_time(q1) / reps
+
+    # ---- in-repo BF16 comparator on the same shapes
+    bf16_ms = None
+    if not args.no_bf16:
+        for _ in range(2):
+            vca.bf16_attention_fwd(Q, K, V, scale, O=O, ws=ws)
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        b0.record(stream)
+        for _ in range(3):
+            vca.bf16_attention_fwd(Q, K, V, scale, O=O, ws=ws)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        bf16_ms = b0.elapsed_time(b1) / 3
+    ws.check()
+
+    # ---- end to end through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+        hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        dQ, dK, dV = (torch.empty_like(t) for t in (Q, K, V))
+
+        def e2e_step():
+            dQ.copy_(hQ, non_blocking=True)
+            dK.copy_(hK, non_blocking=True)
+            dV.copy_(hV, non_blocking=True)
+            _, _, pp = vca.cluster_permute(dV, w.k, KMEANS_ITERS, ws=ws)
+            vca.smooth_quantize(dQ, dK, dV, pp, out=ops, ws=ws)
+            vca.attention_fwd(ops, N, scale, O=O, ws=ws)
+            hO.copy_(O, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(2, min(args.steps, 5))
+        barrier(world)
+        torch.cuda.synchronize()
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        x1.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = max_over_ranks(x0.elapsed_time(x1) / 1e3 / n_e2e, world)
+        e2e = {"value": world * w.flops / t_e2e / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2,
+               "ms_per_step": t_e2e * 1e3}
+        ws.check()
+
+    peaks, peak_kind = load_peaks()
+    fp8_peak_sust = peaks["bf16_tflops_sustained"] * FP8_PER_BF16
+    fp8_peak_burst = peaks["bf16_tflops"] * FP8_PER_BF16
+    achieved = w.flops / t_attn / 1e12
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "attn_fp8_traffic.json")
+    if os.path.exists(tfile):
+        with open(tfile) as f:
+            tj = json.load(f)
+        if tj.get("workload") == args.workload and tj.get("kernel_rev") == kernel_revision():
+            traffic = tj.get("dram_bytes_per_launch")
+    ms_step = t_total / args.steps * 1e3
+    value = world * w.flops / (t_total / args.steps) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3 (fp32 accumulate)",
+        "data": "synthetic (seeded sinusoid video-DiT recipe; see workloads.py)",
+        "config": {"workload": f"cfg{w.cid} {w.name}", "B": B, "H": H, "N": N, "d": d,
+                   "grid": list(w.grid) if w.grid else None, "k": w.k, "kmeans_iters": KMEANS_ITERS,
+                   "step": "cluster_permute + smooth_quantize + attention_fwd",
+                   "l2": "inputs (2.3 GB bf16) exceed the 126 MB L2; no flush",
+                   "parallelism": f"replicas x{world} (independent layers, no collective)"},
+        "attn_ms": round(t_attn * 1e3, 3),
+        "attn_tflops": round(achieved, 2),
+        "prep_ms": round(prep_ms, 3),
+        "quant_only_ms": round(quant_ms, 3),
+        "bf16_attn_ms": round(bf16_ms, 3) if bf16_ms else None,
+        "fp8_over_bf16": round(bf16_ms / (t_attn * 1e3), 3) if bf16_ms else None,
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp8_peak_sust, 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / fp8_peak_sust, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind}: bf16 sustained {peaks['bf16_tflops_sustained']} x "
+                                    f"{FP8_PER_BF16} nominal FP8/BF16",
+                     "frac_of_burst": round(achieved / fp8_peak_burst, 4)},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * (args.steps),
+        "clocks": clk.summary(),
+    }
+    return line, (Q, K, V, w)
+
+
+def kernel_revision() -> str:
+    import hashlib
+    p = os.path.join(ROOT, "bit_attention_video_02_b200", "csrc", "vca_attn_fp8.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
+# ------------------------------------------------------------------ oracle timing
+def _bits(t):
+    return W.bf16_bits(t)
+
+
+def run_oracle_baseline(w, Q, K, V, rows=256):
+    """Times the oracle as it stands on a bounded sample of the workload: head
+    0's full prep and `rows` of its query rows, extrapolated linearly to a full
+    step.  Returns (TFLOP/s, threads used, sample description, step seconds)."""
+    import numpy as np
+    import oracle
+    scale = 1.0 / math.sqrt(w.d)
+    Qb, Kb, Vb = (_bits(t[0, 0]) for t in (Q, K, V))
+    t0 = time.perf_counter()
+    ops = oracle.prep_head(Qb, Kb, Vb, w.k, KMEANS_ITERS)
+    t1 = time.perf_counter()
+    rng = np.random.default_rng(7)
+    rsel = np.sort(rng.choice(w.N, size=min(rows, w.N), replace=False)).astype(np.int32)
+    oracle.attention_head(ops, w.N, scale, rows=rsel)
+    t2 = time.perf_counter()
+    per_head = (t1 - t0) + (t2 - t1) * (w.N / len(rsel))
+    step_s = per_head * w.B * w.H
+    desc = (f"head 0 of cfg{w.cid}: full prep (k-means x{KMEANS_ITERS}, permutation, quantisation) "
+            f"{t1 - t0:.2f}s + attention for {len(rsel)} of {w.N} query rows {t2 - t1:.2f}s; "
+            f"extrapolated linearly to {w.B * w.H} heads x {w.N} rows")
+    return w.flops / step_s / 1e12, oracle.num_threads(), desc, step_s
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = W.WORKLOADS[args.workload]
+    Q, K, V = W.make_qkv(w, "cuda" if torch.cuda.is_available() else "cpu")
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, cores, desc, step_s = run_oracle_baseline(w, Q, K, V, rows=64)
+        if i >= args.warmup:
+            vals.append((v, step_s))
+    value = statistics.mean(v for v, _ in vals)
+    step_ms = statistics.mean(s for _, s in vals) * 1e3
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+        "data": "synthetic (seeded sinusoid video-DiT recipe)",
+        "config": {"workload": f"cfg{w.cid} {w.name}", "B": w.B, "H": w.H, "N": w.N, "d": w.d, "k": w.k},
+        "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": desc, "value": value},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-bf16", action="store_true")
+    args = ap.parse_args()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+        else:
+            line, (Q, K, V, w) = run_ours(args, world, rank, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                v, cores, desc, _ = run_oracle_baseline(w, Q, K, V)
+                line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                        "sample": desc}
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
