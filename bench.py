@@ -140,7 +140,7 @@ class ClockSampler:
 # ------------------------------------------------------------------ our arm
 def run_ours(args, world, rank, local):
     vca_build.build()
-    w = W.WORKLOADS[args.workload]
+    w = W.shrink(W.WORKLOADS[args.workload], H=args.heads)
     dev = torch.device("cuda", local)
     scale = 1.0 / math.sqrt(w.d)
     Q, K, V = W.make_qkv(w, dev)
@@ -336,7 +336,7 @@ def run_oracle_baseline(w, Q, K, V, rows=256):
 def run_reference(args, world, rank):
     if rank != 0:
         return None
-    w = W.WORKLOADS[args.workload]
+    w = W.shrink(W.WORKLOADS[args.workload], H=args.heads)
     Q, K, V = W.make_qkv(w, "cuda" if torch.cuda.is_available() else "cpu")
     vals = []
     for i in range(args.warmup + args.steps):
@@ -363,6 +363,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", type=int, default=3)
+    ap.add_argument("--heads", type=int, default=None, help="run the workload with fewer heads (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bf16", action="store_true")
