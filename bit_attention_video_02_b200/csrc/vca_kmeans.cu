@@ -15,6 +15,8 @@
 // (one fp64 division per centroid coordinate).  Then a stable counting sort:
 // per-chunk histograms, an exclusive scan in (cluster, chunk) order, and a
 // warp-synchronous ranked scatter.
+#include <mutex>
+
 #include "vca_device.cuh"
 #include "vca_host.h"
 
@@ -298,6 +300,64 @@ extern "C" int vca_cluster_permute(const vca_bf16* V, int B, int H, int N, int d
     return fail(VCA_ERR_WORKSPACE, "vca_cluster_permute: workspace needs %zu bytes", need);
   size_t total;
   KmWs w = carve(ws, B * H, N, k, &total);
+  return cluster_permute_impl(V, B, H, N, d, k, iters, init_centroids, centroids, assign, perm, w,
+                              (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------- no-allocation variant
+//
+// Some callers cannot allocate device memory at the moment they run the
+// grouping step: a plugin invoked from an engine that owns and budgets all GPU
+// memory itself, or a latency-critical enqueue path where cudaMalloc may
+// synchronise the device and stall other streams.  For them the scratch lives in
+// one fixed array below, reserved on every GPU that loads this library until the
+// process exits.  All calls share it, so calls whose kernels overlap on the GPU
+// (other streams, other threads) race; serialise them on one stream.
+
+static __device__ __align__(256) unsigned char g_cluster_scratch[VCA_NOALLOC_SCRATCH_BYTES];
+
+// The array's host-side name is only a stand-in for the symbol; the device
+// address comes from cudaGetSymbolAddress, looked up once per device with that
+// device current (the first call on each device does it).
+static int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[256] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(VCA_ERR_CUDA, "vca_cluster_permute_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 256) return fail(VCA_ERR_UNSUPPORTED, "vca_cluster_permute_noalloc: device %d out of range", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_cluster_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(VCA_ERR_CUDA, "vca_cluster_permute_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return VCA_OK;
+}
+
+extern "C" int vca_cluster_permute_noalloc(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
+                                           const float* init_centroids, float* centroids, int32_t* assign,
+                                           int32_t* perm, vca_stream_t stream) {
+  int rc = check_cluster_args(V, B, H, N, d, k, iters, init_centroids, centroids, assign, perm);
+  if (rc) return rc;
+  size_t need = vca_cluster_permute_workspace_size(B, H, N, k);
+  if (need > (size_t)VCA_NOALLOC_SCRATCH_BYTES)
+    return fail(VCA_ERR_UNSUPPORTED,
+                "vca_cluster_permute_noalloc: B=%d H=%d N=%d k=%d needs %zu bytes of scratch, more than the "
+                "fixed %zu; use vca_cluster_permute with a workspace",
+                B, H, N, k, need, (size_t)VCA_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  // the array keeps the previous call's contents: the status word is cleared
+  // here; the sums and counts are cleared before every k-means round and the
+  // sort tables are written in full before they are read
+  if (cudaMemsetAsync(scratch, 0, sizeof(DevStatus), (cudaStream_t)stream) != cudaSuccess)
+    return fail(VCA_ERR_CUDA, "vca_cluster_permute_noalloc: cudaMemsetAsync failed");
+  size_t total;
+  KmWs w = carve(scratch, B * H, N, k, &total);
   return cluster_permute_impl(V, B, H, N, d, k, iters, init_centroids, centroids, assign, perm, w,
                               (cudaStream_t)stream);
 }

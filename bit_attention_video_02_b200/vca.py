@@ -29,7 +29,7 @@ _lib = None
 EXPORTED = [
     "vca_status_bytes", "vca_reset_status", "vca_check_status", "vca_last_error",
     "vca_set_wait_limit_ns", "vca_debug_wait_timeout", "vca_expcast_ref", "vca_e4m3_encode",
-    "vca_cluster_permute_workspace_size", "vca_cluster_permute",
+    "vca_cluster_permute_workspace_size", "vca_cluster_permute", "vca_cluster_permute_noalloc",
     "vca_smooth_quantize_workspace_size", "vca_smooth_quantize_qkv",
     "vca_attention_workspace_size", "vca_attention_fwd",
     "vca_bf16_attention_workspace_size", "vca_bf16_attention_fwd",
@@ -60,6 +60,7 @@ def lib() -> ctypes.CDLL:
         L.vca_cluster_permute_workspace_size.restype = sz
         L.vca_cluster_permute_workspace_size.argtypes = [i32, i32, i32, i32]
         L.vca_cluster_permute.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp, sz, vp]
+        L.vca_cluster_permute_noalloc.argtypes = [vp, i32, i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]
         L.vca_smooth_quantize_workspace_size.restype = sz
         L.vca_smooth_quantize_workspace_size.argtypes = [i32, i32, i32]
         L.vca_smooth_quantize_qkv.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, i32] + [vp] * 7 + [vp, sz, vp]
@@ -70,7 +71,8 @@ def lib() -> ctypes.CDLL:
         L.vca_bf16_attention_workspace_size.argtypes = [i32, i32, i32]
         L.vca_bf16_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
         for fn in ("vca_reset_status", "vca_check_status", "vca_debug_wait_timeout", "vca_expcast_ref",
-                   "vca_e4m3_encode", "vca_cluster_permute", "vca_smooth_quantize_qkv",
+                   "vca_e4m3_encode", "vca_cluster_permute", "vca_cluster_permute_noalloc",
+                   "vca_smooth_quantize_qkv",
                    "vca_attention_fwd", "vca_bf16_attention_fwd"):
             getattr(L, fn).restype = i32
         _lib = L
@@ -157,6 +159,20 @@ def cluster_permute(V: torch.Tensor, k: int, iters: int = 3, init=None, ws: Work
         assert init.shape == (B, H, k, d) and init.dtype == torch.float32 and init.is_contiguous()
     _check(lib().vca_cluster_permute(_ptr(V), B, H, N, d, k, iters, _ptr(init), _ptr(cent), _ptr(assign),
                                      _ptr(perm), ws.ptr, ws.nbytes, _stream(stream)))
+    return cent, assign, perm
+
+
+def cluster_permute_noalloc(V: torch.Tensor, k: int, iters: int = 3, init=None, centroids=None, assign=None,
+                            perm=None, stream=None):
+    """vca_cluster_permute_noalloc: the library allocates nothing (scratch is a
+    fixed array inside the library); the output tensors may be passed in."""
+    B, H, N, d = _bhnd(V)
+    dev = V.device
+    cent = centroids if centroids is not None else torch.empty(B, H, k, d, dtype=torch.float32, device=dev)
+    assign = assign if assign is not None else torch.empty(B, H, N, dtype=torch.int32, device=dev)
+    perm = perm if perm is not None else torch.empty(B, H, N, dtype=torch.int32, device=dev)
+    _check(lib().vca_cluster_permute_noalloc(_ptr(V), B, H, N, d, k, iters, _ptr(init), _ptr(cent),
+                                             _ptr(assign), _ptr(perm), _stream(stream)))
     return cent, assign, perm
 
 

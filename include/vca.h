@@ -123,6 +123,26 @@ int vca_cluster_permute(const vca_bf16* V, int B, int H, int N, int d, int k, in
                         const float* init_centroids, float* centroids, int32_t* assign,
                         int32_t* perm, void* ws, size_t ws_bytes, vca_stream_t stream);
 
+/* Same grouping as vca_cluster_permute for callers that cannot allocate device
+ * memory when they call it (for example a plugin inside an engine that owns the
+ * whole GPU memory budget, or an enqueue path that must not risk the device-wide
+ * synchronisation cudaMalloc can cause).  The pages have no counterpart: this is
+ * a library convenience.  Identical arguments and results, minus the workspace:
+ * scratch is one fixed array of VCA_NOALLOC_SCRATCH_BYTES inside the library,
+ * held on every GPU that loads the library until the process exits.
+ *  - Shapes whose workspace (vca_cluster_permute_workspace_size) exceeds that
+ *    size are rejected with VCA_ERR_UNSUPPORTED; nothing is allocated, ever.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current); make that first call before any stream capture.
+ *  - Every call uses the same array: calls whose work overlaps on the GPU race.
+ *    Issue them on one stream, or serialise them.
+ *  - Device-side errors are recorded in the array's own status word and are not
+ *    reported to the caller. */
+#define VCA_NOALLOC_SCRATCH_BYTES (8u << 20)
+int vca_cluster_permute_noalloc(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
+                                const float* init_centroids, float* centroids, int32_t* assign,
+                                int32_t* perm, vca_stream_t stream);
+
 size_t vca_smooth_quantize_workspace_size(int B, int H, int N);
 
 /* V-Smooth quantisation ([VCA-news] V-Smooth bullet; [VCA-ru] "Решение": the
