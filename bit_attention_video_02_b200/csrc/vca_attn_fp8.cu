@@ -253,7 +253,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     bool have_ref = false;
     float ltot = 0.0f;
     bool ok = true;
+    // the next tile's K scale and V exponent are loaded one tile ahead, off the
+    // critical path of the score -> code computation
+    float ksc_next = __ldg(ksc);
+    int vex_next = __ldg(vex);
     for (int j = 0; j < nkv; ++j) {
+      const float ksc_j = ksc_next;
+      const int vex_j = vex_next;
+      if (j + 1 < nkv) {
+        ksc_next = __ldg(ksc + j + 1);
+        vex_next = __ldg(vex + j + 1);
+      }
       ok = mbar_wait_warp(&bars.s_full[t], j & 1, &abort_s, p.st, lim, 400 + t);
       if (!ok) break;
       tc_fence_after();
@@ -272,10 +282,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         for (int c = 0; c < 128; ++c)
           if (c >= valid) sv[c] = -INFINITY;
       }
-      float mx = sv[0];
+      // row maximum: four independent chains of 3-input max, chain q over the
+      // 32 scores sv[32q .. 32q+31]
+      float mq[4];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, sv[c]);
-      const float cz = cq * __ldg(ksc + j);        // z = s * cz (log2 domain)
+      for (int q = 0; q < 4; ++q) {
+        float m = sv[32 * q];
+#pragma unroll
+        for (int i = 1; i < 31; i += 2) m = fmax3(m, sv[32 * q + i], sv[32 * q + i + 1]);
+        mq[q] = fmaxf(m, sv[32 * q + 31]);
+      }
+      const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+      const float cz = cq * ksc_j;                 // z = s * cz (log2 domain)
       const float c8 = 8.0f * cz;
       const int ntile = (int)ceilf(__fmaf_rn(mx, cz, -0.08125f));
       // the previous PV into O_t (and sP_t, sL_t reads) must be complete before
@@ -294,31 +312,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         nref = ntile;
         rescale = delta > 126 ? 0.0f : __uint_as_float((uint32_t)(127 - delta) << 23);
       }
-      // ExpCast: code = rne(s*c8 + 87 - 8*nref) via the magic-number FMA,
-      // clamped below at 0; p = decode(code) summed exactly as
-      // float(code << 20) * 2^120.
+      // ExpCast: code = rne(s*c8 + 87 - 8*nref) via the magic-number FMA (two
+      // scores per fma.rn.f32x2), clamped below at 0; the decoded probability is
+      // float(code << 20) * 2^120, summed exactly enough in fp32 pairs
       const float badd = kMagic + (float)(87 - 8 * nref);
-      float lsum = 0.0f;
+      const float2 c8x2 = make_float2(c8, c8), baddx2 = make_float2(badd, badd);
+      float2 lsa = make_float2(0.0f, 0.0f), lsb = make_float2(0.0f, 0.0f);
       const uint32_t prow = smem_u32(sP) + r * 128;
 #pragma unroll
       for (int u16 = 0; u16 < 8; ++u16) {
         uint32_t w4[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          uint32_t b[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float f = fmaxf(__fmaf_rn(sv[u16 * 16 + q * 4 + e], c8, badd), kMagic);
-            b[e] = __float_as_uint(f);
-            lsum += __uint_as_float(b[e] << 20);
-          }
-          w4[q] = prmt(prmt(b[0], b[1], 0x0040u), prmt(b[2], b[3], 0x0040u), 0x5410u);
+          const int c = u16 * 16 + q * 4;
+          const float2 f01 = __ffma2_rn(make_float2(sv[c], sv[c + 1]), c8x2, baddx2);
+          const float2 f23 = __ffma2_rn(make_float2(sv[c + 2], sv[c + 3]), c8x2, baddx2);
+          const uint32_t b0 = __float_as_uint(fmaxf(f01.x, kMagic)), b1 = __float_as_uint(fmaxf(f01.y, kMagic));
+          const uint32_t b2 = __float_as_uint(fmaxf(f23.x, kMagic)), b3 = __float_as_uint(fmaxf(f23.y, kMagic));
+          lsa = __fadd2_rn(lsa, make_float2(__uint_as_float(b0 << 20), __uint_as_float(b1 << 20)));
+          lsb = __fadd2_rn(lsb, make_float2(__uint_as_float(b2 << 20), __uint_as_float(b3 << 20)));
+          w4[q] = prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
         }
         const uint32_t addr = prow + ((uint32_t)(u16 ^ (r & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w4[0]), "r"(w4[1]),
                      "r"(w4[2]), "r"(w4[3])
                      : "memory");
       }
+      const float lsum = (lsa.x + lsa.y) + (lsb.x + lsb.y);
       const float l = lsum * 0x1p120f;
       // block row sum -> L tile (hi part exact in TF32, lo the remainder)
       {
@@ -357,7 +377,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       ltot = ltot * rescale + l;
       // UE8M0 scale vectors for this PV: A = 2^0, B = 2^v_exp[j]
       {
-        const uint32_t eb = (uint32_t)(127 + (int)__ldg(vex + j));
+        const uint32_t eb = (uint32_t)(127 + vex_j);
         uint32_t sf[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) sf[i] = 0x7F7F7F7Fu;

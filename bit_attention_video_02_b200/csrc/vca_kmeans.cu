@@ -68,14 +68,23 @@ __global__ void km_init_kernel(const uint16_t* __restrict__ V, const float* __re
   }
 }
 
+// Shared-memory centroid table for the assignment: pairs of centroids
+// interleaved per channel and negated, cs[p][ch] = (-mu_{2p}[ch], -mu_{2p+1}[ch]),
+// so one fma.rn.f32x2 advances the distances to two centroids.  An odd k is
+// padded with a centroid at infinity, which never wins.
 __global__ void __launch_bounds__(kAssignThreads) km_assign_kernel(const uint16_t* __restrict__ V,
                                                                   const float* __restrict__ cent,
                                                                   int32_t* __restrict__ assign,
                                                                   int N, int k) {
-  extern __shared__ float4 cs4[];   // [k][32] float4 = [k][128] floats
+  extern __shared__ float4 cs4[];   // [ceil(k/2)][64] float4 = [pairs][128 channels][2]
   const int bh = blockIdx.y;
-  const float4* src = reinterpret_cast<const float4*>(cent + (int64_t)bh * k * 128);
-  for (int i = threadIdx.x; i < k * 32; i += blockDim.x) cs4[i] = src[i];
+  const int npairs = (k + 1) >> 1;
+  const float* src = cent + (int64_t)bh * k * 128;
+  float2* cs2 = reinterpret_cast<float2*>(cs4);
+  for (int i = threadIdx.x; i < npairs * 128; i += blockDim.x) {
+    const int pp = i >> 7, ch = i & 127, c0 = 2 * pp, c1 = 2 * pp + 1;
+    cs2[i] = make_float2(-src[c0 * 128 + ch], c1 < k ? -src[c1 * 128 + ch] : -INFINITY);
+  }
   __syncthreads();
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
@@ -88,23 +97,25 @@ __global__ void __launch_bounds__(kAssignThreads) km_assign_kernel(const uint16_
   }
   int best = 0;
   float bd = 0.0f;
-  for (int c = 0; c < k; ++c) {
-    const float4* cc = cs4 + c * 32;
-    float acc = 0.0f;
+  for (int pp = 0; pp < npairs; ++pp) {
+    const float4* cc = cs4 + pp * 64;
+    float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      float4 m = cc[i];
-      float x0 = __uint_as_float(v[2 * i] << 16), x1 = __uint_as_float(v[2 * i] & 0xFFFF0000u);
-      float x2 = __uint_as_float(v[2 * i + 1] << 16), x3 = __uint_as_float(v[2 * i + 1] & 0xFFFF0000u);
-      float t0 = __fsub_rn(x0, m.x), t1 = __fsub_rn(x1, m.y), t2 = __fsub_rn(x2, m.z), t3 = __fsub_rn(x3, m.w);
-      acc = __fmaf_rn(t0, t0, acc);
-      acc = __fmaf_rn(t1, t1, acc);
-      acc = __fmaf_rn(t2, t2, acc);
-      acc = __fmaf_rn(t3, t3, acc);
+    for (int i = 0; i < 64; ++i) {
+      const float4 m = cc[i];            // channels 2i (x, y) and 2i+1 (z, w)
+      const float x0 = __uint_as_float(v[i] << 16), x1 = __uint_as_float(v[i] & 0xFFFF0000u);
+      float2 t = __fadd2_rn(make_float2(x0, x0), make_float2(m.x, m.y));   // v - mu, exact order per lane
+      acc = __ffma2_rn(t, t, acc);
+      t = __fadd2_rn(make_float2(x1, x1), make_float2(m.z, m.w));
+      acc = __ffma2_rn(t, t, acc);
     }
-    if (c == 0 || acc < bd) {
-      bd = acc;
-      best = c;
+    if (pp == 0 || acc.x < bd) {
+      bd = acc.x;
+      best = 2 * pp;
+    }
+    if (acc.y < bd) {
+      bd = acc.y;
+      best = 2 * pp + 1;
     }
   }
   assign[(int64_t)bh * N + n] = best;
@@ -126,11 +137,24 @@ __global__ void __launch_bounds__(128) km_accum_kernel(const uint16_t* __restric
   const int n0 = blockIdx.x * kAccumChunk, n1 = min(N, n0 + kAccumChunk);
   const uint16_t* vb = V + (int64_t)bh * N * 128;
   const int32_t* ab = assign + (int64_t)bh * N;
-  for (int n = n0; n < n1; ++n) {
-    int a = __ldg(ab + n);
-    float v = __uint_as_float((uint32_t)__ldg(vb + (int64_t)n * 128 + ch) << 16);
-    acc[a * 128 + ch] += __float2ll_rn(v * 16777216.0f);
-    if (ch == 0) cnt[a] += 1;
+  // 16 tokens per batch: their loads are independent and overlap
+  for (int nb0 = n0; nb0 < n1; nb0 += 16) {
+    int a[16];
+    uint16_t x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int n = min(nb0 + i, n1 - 1);
+      a[i] = __ldg(ab + n);
+      x[i] = __ldg(vb + (int64_t)n * 128 + ch);
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (nb0 + i < n1) {
+        const float v = __uint_as_float((uint32_t)x[i] << 16);
+        acc[a[i] * 128 + ch] += __float2ll_rn(v * 16777216.0f);
+        if (ch == 0) cnt[a[i]] += 1;
+      }
+    }
   }
   __syncthreads();
   long long* dst = sums + (int64_t)bh * k * 128;
@@ -247,7 +271,7 @@ static int cluster_permute_impl(const vca_bf16* V, int B, int H, int N, int d, i
   km_init_kernel<<<dim3(BH, k), 128, 0, s>>>(V, init, cent, N, k);
   int rc = check_launch("km_init_kernel");
   if (rc) return rc;
-  const size_t assign_smem = (size_t)k * 128 * sizeof(float);
+  const size_t assign_smem = (size_t)((k + 1) / 2) * 128 * sizeof(float2);
   const size_t accum_smem = (size_t)k * 128 * sizeof(long long);
   if (cudaFuncSetAttribute(km_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)assign_smem) !=
           cudaSuccess ||

@@ -7,7 +7,8 @@
 // mean is stored exactly; "Nunchux AI Introduces VC-Attention..." (abstract):
 // a mean costs 0.125 bit per value element (16 bits per 128 tokens).
 //
-// One CTA per (128-token block, tensor, head): 256 threads, HBM-bound.  Loads
+// One CTA per (128-token block, tensor, head): 256 threads, HBM-bound; Q/K and
+// V blocks are two launches of the same kernel (only V uses shared memory).  Loads
 // are 16-byte vectors of whole token rows (gathered through the permutation for
 // K and V); Q/K codes are written straight from registers, the V residual is
 // transposed through shared memory so VrT rows (channel-major) are written as
@@ -35,6 +36,7 @@ struct PrepArgs {
   int8_t* v_exp;
   uint16_t* v_mean;
   DevStatus* st;
+  int tensor_base;   // blockIdx.y + tensor_base: 0 = Q, 1 = K, 2 = V
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -99,7 +101,7 @@ __global__ void __launch_bounds__(kPrepThreads) smooth_quant_kernel(const PrepAr
   __shared__ float mu_s[128];
   __shared__ int flag_s;
 
-  const int blk = blockIdx.x, tensor = blockIdx.y, bh = blockIdx.z;
+  const int blk = blockIdx.x, tensor = blockIdx.y + a.tensor_base, bh = blockIdx.z;
   const int N = a.N, nb = a.nb;
   const int64_t Np = (int64_t)nb * 128;
   const int n0 = blk * 128;
@@ -269,7 +271,13 @@ extern "C" int vca_smooth_quantize_qkv(const vca_bf16* Q, const vca_bf16* K, con
   a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.N = N; a.nb = (N + 127) / 128;
   a.Qq = Qq; a.q_scale = q_scale; a.Kq = Kq; a.k_scale = k_scale; a.VrT = VrT;
   a.v_exp = v_exp; a.v_mean = v_mean; a.st = (DevStatus*)ws;
-  dim3 grid(a.nb, 3, B * H);
-  smooth_quant_kernel<<<grid, kPrepThreads, kPrepSmem, (cudaStream_t)stream>>>(a);
-  return check_launch("smooth_quant_kernel");
+  // Q and K blocks need no shared tile: a launch of their own keeps them at full
+  // occupancy; the V blocks (mean, residual, transpose) get the shared tile
+  a.tensor_base = 0;
+  smooth_quant_kernel<<<dim3(a.nb, 2, B * H), kPrepThreads, 0, (cudaStream_t)stream>>>(a);
+  int rc = check_launch("smooth_quant_kernel (Q, K)");
+  if (rc) return rc;
+  a.tensor_base = 2;
+  smooth_quant_kernel<<<dim3(a.nb, 1, B * H), kPrepThreads, kPrepSmem, (cudaStream_t)stream>>>(a);
+  return check_launch("smooth_quant_kernel (V)");
 }
