@@ -15,11 +15,13 @@
 //    warpgroups of query tile 0 / 1 (thread = query row = TMEM lane).
 //  * TMEM (512 columns): S0, S1 (fp32 scores), O0, O1 (fp32 accumulators).
 //  * S_t = Q_t K_j^T: tcgen05 kind::f8f6f4, operands from 128B-swizzled smem.
-//  * O_t += P_t R_j * 2^e_j: kind::mxf8f6f4.block_scale; the per-block V
-//    exponent is the UE8M0 scale of B (A's scale is 1).  The two 4-column scale
-//    vectors are written into the already-consumed S_t columns, so the next
-//    QK^T (issued after this PV, and tensor-core ops run in issue order)
-//    overwrites them only after they were read.
+//  * O_t += P_t R_j * 2^e_j: kind::mxf8f6f4.block_scale with A = P_t read
+//    from tensor memory (no shared-memory round trip for the probabilities);
+//    the per-block V exponent is the UE8M0 scale of B (A's scale is 1).  P_t
+//    (32 columns of packed E4M3 codes) and the two 4-column scale vectors are
+//    written into the already-consumed S_t columns, so the next QK^T (issued
+//    after this PV; tensor-core ops run in issue order) overwrites them only
+//    after they were read.
 //  * Mean restore: every 8 key blocks, O_t += L_t M^T with a TF32 MMA, where
 //    L_t[i][b] are the block row sums (split hi + lo so they keep ~22 bits) and
 //    M[d][b] the bf16 block means (exact in TF32).
@@ -45,8 +47,7 @@ constexpr int kGroup = 8;   // key blocks per mean-restore MMA
 constexpr uint32_t kOffQ = 0;                         // 2 x 16 KB
 constexpr uint32_t kOffK = 32768;                     // kStages x 16 KB
 constexpr uint32_t kOffV = kOffK + kStages * 16384;   // kStages x 16 KB
-constexpr uint32_t kOffP = kOffV + kStages * 16384;   // 2 x 16 KB
-constexpr uint32_t kOffL = kOffP + 32768;             // 2 tiles x (hi 4 KB + lo 4 KB)
+constexpr uint32_t kOffL = kOffV + kStages * 16384;   // 2 tiles x (hi 4 KB + lo 4 KB)
 constexpr uint32_t kOffMu = kOffL + 16384;            // 2 buffers x 4 KB
 constexpr uint32_t kSmemBytes = kOffMu + 8192;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
@@ -162,7 +163,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       const uint32_t id_pv = instr_desc_mx(kFmtE4M3, kFmtE4M3, 128, 128);
       const uint32_t id_mu = instr_desc(kFmtTF32, kFmtTF32, 128, 128, 0, 0);
       const uint32_t sQ = smem_u32(sm + kOffQ), sK = smem_u32(sm + kOffK), sV = smem_u32(sm + kOffV);
-      const uint32_t sP = smem_u32(sm + kOffP), sL = smem_u32(sm + kOffL), sMu = smem_u32(sm + kOffMu);
+      const uint32_t sL = smem_u32(sm + kOffL), sMu = smem_u32(sm + kOffMu);
       bool ok = mbar_wait_bounded(&bars.q_full, 0, &abort_s, p.st, lim, 200);
       ok = ok && mbar_wait_bounded(&bars.kv_full[0], 0, &abort_s, p.st, lim, 201);
       if (ok) {
@@ -183,8 +184,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
           if (!ok) break;
           tc_fence_after();
           const uint32_t sft = tmem + t * 128;   // scale vectors live in the consumed S_t columns
-          for (int k = 0; k < 4; ++k)
-            mma_mxf8_ss(tmem + 256 + t * 128, smem_desc(sP + t * 16384 + 32 * k, 16, 1024, kLayoutSW128),
+          for (int k = 0; k < 4; ++k)   // P_t at S_t columns 8..39, 8 columns (32 codes) per K step
+            mma_mxf8_ts(tmem + 256 + t * 128, sft + 8 + 8 * k,
                         smem_desc(sV + s * 16384 + 32 * k, 16, 1024, kLayoutSW128), id_pv, sft, sft + 4,
                         (j > 0 || k > 0) ? 1u : 0u);
           if (group_end) {
@@ -245,7 +246,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const float sq = qvalid ? __ldg(p.q_scale + (int64_t)bh * nb + qtile) : 1.0f;
     const float cq = sq * p.c_base;
     const float kMagic = 12582912.0f;              // 1.5 * 2^23: adding it rounds to an integer
-    uint8_t* sP = sm + kOffP + t * 16384;
     uint8_t* sLt = sm + kOffL + t * 8192;
     const float* ksc = p.k_scale + (int64_t)bh * nb;
     const int8_t* vex = p.v_exp + (int64_t)bh * nb;
@@ -296,13 +296,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       const float cz = cq * ksc_j;                 // z = s * cz (log2 domain)
       const float c8 = 8.0f * cz;
       const int ntile = (int)ceilf(__fmaf_rn(mx, cz, -0.08125f));
-      // the previous PV into O_t (and sP_t, sL_t reads) must be complete before
-      // O_t is rescaled or sP_t / sL_t are overwritten
-      if (j > 0) {
-        ok = mbar_wait_warp(&bars.o_done[t], (j - 1) & 1, &abort_s, p.st, lim, 410 + t);
-        if (!ok) break;
-        tc_fence_after();
-      }
+      // (S_t(j) was committed after PV_t(j-1) and any mean MMA before it, so
+      // those have completed: O_t may be rescaled and sL_t rewritten now)
       float rescale = 1.0f;       // O_t and the pending row sums are scaled by this
       if (!have_ref) {
         nref = ntile;
@@ -318,26 +313,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       const float badd = kMagic + (float)(87 - 8 * nref);
       const float2 c8x2 = make_float2(c8, c8), baddx2 = make_float2(badd, badd);
       float2 lsa = make_float2(0.0f, 0.0f), lsb = make_float2(0.0f, 0.0f);
-      const uint32_t prow = smem_u32(sP) + r * 128;
+      uint32_t pw[32];   // the row's 128 codes, 4 per word, in key order
 #pragma unroll
-      for (int u16 = 0; u16 < 8; ++u16) {
-        uint32_t w4[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c = u16 * 16 + q * 4;
-          const float2 f01 = __ffma2_rn(make_float2(sv[c], sv[c + 1]), c8x2, baddx2);
-          const float2 f23 = __ffma2_rn(make_float2(sv[c + 2], sv[c + 3]), c8x2, baddx2);
-          const uint32_t b0 = __float_as_uint(fmaxf(f01.x, kMagic)), b1 = __float_as_uint(fmaxf(f01.y, kMagic));
-          const uint32_t b2 = __float_as_uint(fmaxf(f23.x, kMagic)), b3 = __float_as_uint(fmaxf(f23.y, kMagic));
-          lsa = __fadd2_rn(lsa, make_float2(__uint_as_float(b0 << 20), __uint_as_float(b1 << 20)));
-          lsb = __fadd2_rn(lsb, make_float2(__uint_as_float(b2 << 20), __uint_as_float(b3 << 20)));
-          w4[q] = prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
-        }
-        const uint32_t addr = prow + ((uint32_t)(u16 ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w4[0]), "r"(w4[1]),
-                     "r"(w4[2]), "r"(w4[3])
-                     : "memory");
+      for (int q = 0; q < 32; ++q) {
+        const int c = q * 4;
+        const float2 f01 = __ffma2_rn(make_float2(sv[c], sv[c + 1]), c8x2, baddx2);
+        const float2 f23 = __ffma2_rn(make_float2(sv[c + 2], sv[c + 3]), c8x2, baddx2);
+        const uint32_t b0 = __float_as_uint(fmaxf(f01.x, kMagic)), b1 = __float_as_uint(fmaxf(f01.y, kMagic));
+        const uint32_t b2 = __float_as_uint(fmaxf(f23.x, kMagic)), b3 = __float_as_uint(fmaxf(f23.y, kMagic));
+        lsa = __fadd2_rn(lsa, make_float2(__uint_as_float(b0 << 20), __uint_as_float(b1 << 20)));
+        lsb = __fadd2_rn(lsb, make_float2(__uint_as_float(b2 << 20), __uint_as_float(b3 << 20)));
+        pw[q] = prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
       }
+      VCA_TMEM_ST32(tS + 8, pw);
       const float lsum = (lsa.x + lsa.y) + (lsb.x + lsb.y);
       const float l = lsum * 0x1p120f;
       // block row sum -> L tile (hi part exact in TF32, lo the remainder)
