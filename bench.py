@@ -74,6 +74,12 @@ def barrier(world):
         dist.barrier()
 
 
+def whole_job_value(world: int, flops_per_rank: float, seconds_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank runs its own layer of `flops_per_rank`
+    (weak scaling) and the step time is the slowest rank's."""
+    return world * flops_per_rank / seconds_per_step / 1e12
+
+
 def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
@@ -243,7 +249,7 @@ def run_ours(args, world, rank, local):
         x1.record(stream)
         torch.cuda.synchronize()
         t_e2e = max_over_ranks(x0.elapsed_time(x1) / 1e3 / n_e2e, world)
-        e2e = {"value": world * w.flops / t_e2e / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": whole_job_value(world, w.flops, t_e2e), "unit": "TFLOP/s",
                "h2d_bytes_per_step": 3 * Q.numel() * 2, "d2h_bytes_per_step": O.numel() * 2,
                "ms_per_step": t_e2e * 1e3}
         ws.check()
@@ -260,7 +266,7 @@ def run_ours(args, world, rank, local):
         if tj.get("workload") == args.workload and tj.get("kernel_rev") == kernel_revision():
             traffic = tj.get("dram_bytes_per_launch")
     ms_step = t_total / args.steps * 1e3
-    value = world * w.flops / (t_total / args.steps) / 1e12
+    value = whole_job_value(world, w.flops, t_total / args.steps)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -369,6 +375,8 @@ def main():
     ap.add_argument("--no-bf16", action="store_true")
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
+    if args.gpus != world and rank == 0:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; reporting {world} rank(s)", file=sys.stderr)
     try:
         if args.impl == "reference":
             line = run_reference(args, world, rank)
