@@ -158,64 +158,74 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t id_qk = instr_desc(kFmtE4M3, kFmtE4M3, 128, 128, 0, 0);
-      const uint32_t id_pv = instr_desc_mx(kFmtE4M3, kFmtE4M3, 128, 128);
-      const uint32_t id_mu = instr_desc(kFmtTF32, kFmtTF32, 128, 128, 0, 0);
-      const uint32_t sQ = smem_u32(sm + kOffQ), sK = smem_u32(sm + kOffK), sV = smem_u32(sm + kOffV);
-      const uint32_t sL = smem_u32(sm + kOffL), sMu = smem_u32(sm + kOffMu);
-      bool ok = mbar_wait_bounded(&bars.q_full, 0, &abort_s, p.st, lim, 200);
-      ok = ok && mbar_wait_bounded(&bars.kv_full[0], 0, &abort_s, p.st, lim, 201);
-      if (ok) {
-        tc_fence_after();
-        for (int t = 0; t < 2; ++t) {
-          for (int k = 0; k < 4; ++k)
-            mma_f8_ss(tmem + t * 128, smem_desc(sQ + t * 16384 + 32 * k, 16, 1024, kLayoutSW128),
-                      smem_desc(sK + 32 * k, 16, 1024, kLayoutSW128), id_qk, k > 0);
-          tc_commit(&bars.s_full[t]);
-        }
+    // The whole warp runs this loop in lockstep, so descriptors are computed
+    // once, stay warp-uniform and advance by constants; one elected lane issues
+    // each tcgen05 instruction.  (The issuing warp shares its SM sub-partition
+    // with two softmax warps: the fewer instructions per MMA, the sooner the
+    // tensor pipe gets its next operation.)
+    const uint32_t id_qk = instr_desc(kFmtE4M3, kFmtE4M3, 128, 128, 0, 0);
+    const uint32_t id_pv = instr_desc_mx(kFmtE4M3, kFmtE4M3, 128, 128);
+    const uint32_t id_mu = instr_desc(kFmtTF32, kFmtTF32, 128, 128, 0, 0);
+    // descriptor start addresses count 16-byte units: +2 per 32-byte K step,
+    // +1024 per 16 KB tile, +256 per 4 KB
+    const uint64_t dQ = smem_desc(smem_u32(sm + kOffQ), 16, 1024, kLayoutSW128);
+    const uint64_t dK = smem_desc(smem_u32(sm + kOffK), 16, 1024, kLayoutSW128);
+    const uint64_t dV = smem_desc(smem_u32(sm + kOffV), 16, 1024, kLayoutSW128);
+    const uint64_t dL = smem_desc(smem_u32(sm + kOffL), 128, 256, kLayoutNone);
+    const uint64_t dMu = smem_desc(smem_u32(sm + kOffMu), 128, 256, kLayoutNone);
+    bool ok = mbar_wait_warp(&bars.q_full, 0, &abort_s, p.st, lim, 200);
+    ok = ok && mbar_wait_warp(&bars.kv_full[0], 0, &abort_s, p.st, lim, 201);
+    if (ok) {
+      tc_fence_after();
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_f8_ss_w(tmem + t * 128, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(2 * k), id_qk, k > 0);
+        tc_commit_w(&bars.s_full[t]);
       }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % kStages;
-        const bool group_end = (j % kGroup == kGroup - 1) || (j == nkv - 1);
-        const int g = j / kGroup, gb = g & 1;
-        for (int t = 0; t < 2 && ok; ++t) {
-          ok = mbar_wait_bounded(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t);
+    }
+    for (int j = 0; ok && j < nkv; ++j) {
+      const int s = j % kStages;
+      const bool group_end = (j % kGroup == kGroup - 1) || (j == nkv - 1);
+      const int g = j / kGroup, gb = g & 1;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        ok = mbar_wait_warp(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t sft = tmem + t * 128;   // scale vectors live in the consumed S_t columns
+#pragma unroll
+        for (int k = 0; k < 4; ++k)   // P_t at S_t columns 8..39, 8 columns (32 codes) per K step
+          mma_mxf8_ts_w(tmem + 256 + t * 128, sft + 8 + 8 * k, dV + (uint64_t)(s * 1024 + 2 * k), id_pv, sft,
+                        sft + 4, (j > 0 || k > 0) ? 1u : 0u);
+        if (group_end) {
+          ok = mbar_wait_warp(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t sft = tmem + t * 128;   // scale vectors live in the consumed S_t columns
-          for (int k = 0; k < 4; ++k)   // P_t at S_t columns 8..39, 8 columns (32 codes) per K step
-            mma_mxf8_ts(tmem + 256 + t * 128, sft + 8 + 8 * k,
-                        smem_desc(sV + s * 16384 + 32 * k, 16, 1024, kLayoutSW128), id_pv, sft, sft + 4,
-                        (j > 0 || k > 0) ? 1u : 0u);
-          if (group_end) {
-            ok = mbar_wait_bounded(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220);
+          const uint64_t bdesc = dMu + (uint64_t)(gb * 256);
+          mma_tf32_ss_w(tmem + 256 + t * 128, dL + (uint64_t)(t * 512), bdesc, id_mu, 1u);
+          mma_tf32_ss_w(tmem + 256 + t * 128, dL + (uint64_t)(t * 512 + 256), bdesc, id_mu, 1u);
+          if (t == 1) tc_commit_w(&bars.mu_empty[gb]);
+        }
+        tc_commit_w(&bars.o_done[t]);
+        if (t == 1) tc_commit_w(&bars.kv_empty[s]);
+        if (j + 1 < nkv) {
+          const int s1 = (j + 1) % kStages;
+          if (t == 0) {
+            ok = mbar_wait_warp(&bars.kv_full[s1], ((j + 1) / kStages) & 1, &abort_s, p.st, lim, 230);
             if (!ok) break;
             tc_fence_after();
-            const uint64_t bdesc = smem_desc(sMu + gb * 4096, 128, 256, kLayoutNone);
-            mma_tf32_ss(tmem + 256 + t * 128, smem_desc(sL + t * 8192, 128, 256, kLayoutNone), bdesc, id_mu, 1u);
-            mma_tf32_ss(tmem + 256 + t * 128, smem_desc(sL + t * 8192 + 4096, 128, 256, kLayoutNone), bdesc,
-                        id_mu, 1u);
-            if (t == 1) tc_commit(&bars.mu_empty[gb]);
           }
-          tc_commit(&bars.o_done[t]);
-          if (t == 1) tc_commit(&bars.kv_empty[s]);
-          if (j + 1 < nkv) {
-            const int s1 = (j + 1) % kStages;
-            if (t == 0) {
-              ok = mbar_wait_bounded(&bars.kv_full[s1], ((j + 1) / kStages) & 1, &abort_s, p.st, lim, 230);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            for (int k = 0; k < 4; ++k)
-              mma_f8_ss(tmem + t * 128, smem_desc(sQ + t * 16384 + 32 * k, 16, 1024, kLayoutSW128),
-                        smem_desc(sK + s1 * 16384 + 32 * k, 16, 1024, kLayoutSW128), id_qk, k > 0);
-            tc_commit(&bars.s_full[t]);
-          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_f8_ss_w(tmem + t * 128, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(s1 * 1024 + 2 * k),
+                        id_qk, k > 0);
+          tc_commit_w(&bars.s_full[t]);
         }
       }
-      tc_commit(&bars.mma_done);
     }
+    tc_commit_w(&bars.mma_done);
   } else if (warp == 2) {
     // ------------------------------------------------------------ block means -> fp32 [d][8] tiles
     const uint16_t* vm = p.v_mean + (int64_t)bh * nb * 128;

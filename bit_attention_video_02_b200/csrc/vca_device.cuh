@@ -210,6 +210,41 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d, uint32_t a_tmem, uint64_t 
       "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum));
 }
 
+// Warp-issued forms: the whole converged warp runs the issue loop in lockstep
+// (so descriptors and addresses stay warp-uniform and cost one set of uniform
+// instructions) and elect.sync picks the issuing lane -- lane 0 whenever all 32
+// lanes are active, so MMAs and the commits that track them come from the same
+// thread.
+__device__ __forceinline__ void mma_f8_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+__device__ __forceinline__ void mma_mxf8_ts_w(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                              uint32_t sfa, uint32_t sfb, uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %6, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], [%1], %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accum));
+}
+__device__ __forceinline__ void mma_tf32_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                              uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
+__device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 // 32 consecutive 32-bit TMEM columns of this thread's lane -> registers.
 #define VCA_TMEM_LD32(taddr, r)                                                                  \
   asm volatile(                                                                                  \
