@@ -71,98 +71,180 @@ __global__ void km_init_kernel(const uint16_t* __restrict__ V, const float* __re
 // Shared-memory centroid table for the assignment: pairs of centroids
 // interleaved per channel and negated, cs[p][ch] = (-mu_{2p}[ch], -mu_{2p+1}[ch]),
 // so one fma.rn.f32x2 advances the distances to two centroids.  An odd k is
-// padded with a centroid at infinity, which never wins.
+// padded with a centroid at infinity, which never wins.  The channel loop is
+// outside the centroid loop, so each bf16 channel is unpacked once per token
+// and feeds NP accumulator pairs; every accumulator still adds its channels
+// in order 0..127 (the distance's defined summation order).
+template <int NP>
 __global__ void __launch_bounds__(kAssignThreads) km_assign_kernel(const uint16_t* __restrict__ V,
                                                                   const float* __restrict__ cent,
                                                                   int32_t* __restrict__ assign,
                                                                   int N, int k) {
-  extern __shared__ float4 cs4[];   // [ceil(k/2)][64] float4 = [pairs][128 channels][2]
+  extern __shared__ float4 cs4[];   // [NP][64] float4 = [pairs][128 channels][2]
   const int bh = blockIdx.y;
   const int npairs = (k + 1) >> 1;
   const float* src = cent + (int64_t)bh * k * 128;
   float2* cs2 = reinterpret_cast<float2*>(cs4);
-  for (int i = threadIdx.x; i < npairs * 128; i += blockDim.x) {
+  for (int i = threadIdx.x; i < NP * 128; i += blockDim.x) {
     const int pp = i >> 7, ch = i & 127, c0 = 2 * pp, c1 = 2 * pp + 1;
-    cs2[i] = make_float2(-src[c0 * 128 + ch], c1 < k ? -src[c1 * 128 + ch] : -INFINITY);
+    cs2[i] = make_float2(c0 < k ? -src[c0 * 128 + ch] : -INFINITY, c1 < k ? -src[c1 * 128 + ch] : -INFINITY);
   }
   __syncthreads();
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  // two tokens per thread (n and n + blockDim.x): every centroid value read from
+  // shared memory serves both
+  const int n = blockIdx.x * 2 * blockDim.x + threadIdx.x, nb2 = n + blockDim.x;
   if (n >= N) return;
-  uint32_t v[64];
+  const bool has_b = nb2 < N;
   const uint4* row = reinterpret_cast<const uint4*>(V + ((int64_t)bh * N + n) * 128);
+  const uint4* rowb = reinterpret_cast<const uint4*>(V + ((int64_t)bh * N + (has_b ? nb2 : n)) * 128);
+  float2 acc[NP], accb[NP];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    uint4 q = __ldg(row + i);
-    v[4 * i] = q.x; v[4 * i + 1] = q.y; v[4 * i + 2] = q.z; v[4 * i + 3] = q.w;
-  }
-  int best = 0;
-  float bd = 0.0f;
-  for (int pp = 0; pp < npairs; ++pp) {
-    const float4* cc = cs4 + pp * 64;
-    float2 acc = make_float2(0.0f, 0.0f);
+  for (int pp = 0; pp < NP; ++pp) acc[pp] = accb[pp] = make_float2(0.0f, 0.0f);
+  // 8 channels per step; the next 16-byte pieces of the rows are loaded one step ahead
+  uint4 cur = __ldg(row), curb = __ldg(rowb);
+#pragma unroll 1
+  for (int q = 0; q < 16; ++q) {
+    const int qn = q + 1 < 16 ? q + 1 : q;
+    const uint4 nxt = __ldg(row + qn), nxtb = __ldg(rowb + qn);
+    const uint32_t w[4] = {cur.x, cur.y, cur.z, cur.w}, wb[4] = {curb.x, curb.y, curb.z, curb.w};
 #pragma unroll
-    for (int i = 0; i < 64; ++i) {
-      const float4 m = cc[i];            // channels 2i (x, y) and 2i+1 (z, w)
-      const float x0 = __uint_as_float(v[i] << 16), x1 = __uint_as_float(v[i] & 0xFFFF0000u);
-      float2 t = __fadd2_rn(make_float2(x0, x0), make_float2(m.x, m.y));   // v - mu, exact order per lane
-      acc = __ffma2_rn(t, t, acc);
-      t = __fadd2_rn(make_float2(x1, x1), make_float2(m.z, m.w));
-      acc = __ffma2_rn(t, t, acc);
+    for (int u = 0; u < 4; ++u) {
+      const int i = 4 * q + u;   // channels 2i, 2i+1
+      const float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xFFFF0000u);
+      const float y0 = __uint_as_float(wb[u] << 16), y1 = __uint_as_float(wb[u] & 0xFFFF0000u);
+      const float2 X0 = make_float2(x0, x0), X1 = make_float2(x1, x1);
+      const float2 Y0 = make_float2(y0, y0), Y1 = make_float2(y1, y1);
+#pragma unroll
+      for (int pp = 0; pp < NP; ++pp) {
+        const float4 m = cs4[pp * 64 + i];   // channels 2i (x, y) and 2i+1 (z, w)
+        const float2 m0 = make_float2(m.x, m.y), m1 = make_float2(m.z, m.w);
+        float2 t = __fadd2_rn(X0, m0);   // v - mu, exact order per lane
+        acc[pp] = __ffma2_rn(t, t, acc[pp]);
+        t = __fadd2_rn(X1, m1);
+        acc[pp] = __ffma2_rn(t, t, acc[pp]);
+        t = __fadd2_rn(Y0, m0);
+        accb[pp] = __ffma2_rn(t, t, accb[pp]);
+        t = __fadd2_rn(Y1, m1);
+        accb[pp] = __ffma2_rn(t, t, accb[pp]);
+      }
     }
-    if (pp == 0 || acc.x < bd) {
-      bd = acc.x;
+    cur = nxt;
+    curb = nxtb;
+  }
+  int best = 0, bestb = 0;
+  float bd = acc[0].x, bdb = accb[0].x;
+#pragma unroll
+  for (int pp = 0; pp < NP; ++pp) {
+    if (pp > 0 && acc[pp].x < bd) {
+      bd = acc[pp].x;
       best = 2 * pp;
     }
-    if (acc.y < bd) {
-      bd = acc.y;
+    if (acc[pp].y < bd) {
+      bd = acc[pp].y;
       best = 2 * pp + 1;
     }
+    if (pp > 0 && accb[pp].x < bdb) {
+      bdb = accb[pp].x;
+      bestb = 2 * pp;
+    }
+    if (accb[pp].y < bdb) {
+      bdb = accb[pp].y;
+      bestb = 2 * pp + 1;
+    }
   }
+  if (has_b) assign[(int64_t)bh * N + nb2] = bestb;
+  (void)npairs;
   assign[(int64_t)bh * N + n] = best;
 }
 
-// Exact fixed-point sums per (cluster, channel) for one chunk of tokens; one
-// thread per channel walks the chunk in order (no atomics in shared memory),
-// then the chunk's partial sums are added to the head's totals.
-__global__ void __launch_bounds__(128) km_accum_kernel(const uint16_t* __restrict__ V,
-                                                      const int32_t* __restrict__ assign,
-                                                      long long* __restrict__ sums,
-                                                      int* __restrict__ counts, int N, int k) {
-  extern __shared__ long long acc[];   // [k][128]
+// Exact fixed-point sums per (cluster, channel) for one chunk of tokens.
+// Each warp takes one token at a time, lane l holding channels l + 32j.  The fixed-point value llrint(v * 2^24)
+// (|v| < 2^20, so it has at most 45 bits) is split exactly as hi * 2^22 + lo
+// with |hi|, |lo| < 2^22 using float operations only: f = v * 2^24 is exact,
+// hi = trunc(f / 2^22), lo = rne(f - hi * 2^22) (the only rounding, the same
+// as llrint's), each turned into an integer with the magic-number add.  The
+// halves go into 32-bit shared tables with shared-memory atomics; after every
+// 512 tokens (|sum| < 512 * 2^22 = 2^31, no overflow) they are folded into
+// int64 totals.  Integer addition is exact and order-free, so the result is
+// the exact sum whatever order the warps run in.
+constexpr int kAccumWarps = 8;
+constexpr int kAccumSub = 512;   // tokens between folds of the 32-bit halves
+__device__ __forceinline__ void fix24_split(float v, int& hi, int& lo) {
+  const float kMagic = 12582912.0f;   // 1.5 * 2^23
+  const float f = v * 16777216.0f;
+  const float hf = truncf(f * 2.384185791015625e-07f);     // f / 2^22, truncated
+  const float lf = __fmaf_rn(hf, -4194304.0f, f);         // exact remainder
+  hi = (int)(__float_as_uint(hf + kMagic) - 0x4B400000u);
+  lo = (int)(__float_as_uint(lf + kMagic) - 0x4B400000u);
+}
+__global__ void __launch_bounds__(kAccumWarps * 32) km_accum_kernel(const uint16_t* __restrict__ V,
+                                                                   const int32_t* __restrict__ assign,
+                                                                   long long* __restrict__ sums,
+                                                                   int* __restrict__ counts, int N, int k) {
+  extern __shared__ long long tot[];   // [k][128] int64, then hi[k][128], lo[k][128] int32
+  int* shi = reinterpret_cast<int*>(tot + k * 128);
+  int* slo = shi + k * 128;
   __shared__ int cnt[VCA_MAX_CLUSTERS];
-  const int bh = blockIdx.y, ch = threadIdx.x;
-  for (int c = 0; c < k; ++c) acc[c * 128 + ch] = 0;
-  if (ch < k) cnt[ch] = 0;
+  const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < k * 128; i += blockDim.x) {
+    tot[i] = 0;
+    shi[i] = 0;
+    slo[i] = 0;
+  }
+  if (threadIdx.x < k) cnt[threadIdx.x] = 0;
   __syncthreads();
   const int n0 = blockIdx.x * kAccumChunk, n1 = min(N, n0 + kAccumChunk);
   const uint16_t* vb = V + (int64_t)bh * N * 128;
   const int32_t* ab = assign + (int64_t)bh * N;
-  // 16 tokens per batch: their loads are independent and overlap
-  for (int nb0 = n0; nb0 < n1; nb0 += 16) {
-    int a[16];
-    uint16_t x[16];
+  for (int s0 = n0; s0 < n1; s0 += kAccumSub) {
+    const int s1 = min(n1, s0 + kAccumSub);
+    // two tokens per warp per step so that their loads overlap; lane l takes
+    // channels l, l+32, l+64, l+96 (64-byte coalesced loads, and the shared
+    // tables are hit one bank per lane)
+    for (int n = s0 + warp; n < s1; n += 2 * kAccumWarps) {
+      const int nbk = n + kAccumWarps;
+      const bool hb = nbk < s1;
+      const int a0 = __ldg(ab + n), a1 = hb ? __ldg(ab + nbk) : 0;
+      const uint16_t* r0 = vb + (int64_t)n * 128 + lane;
+      const uint16_t* r1 = vb + (int64_t)(hb ? nbk : n) * 128 + lane;
+      uint16_t x0[4], x1[4];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int n = min(nb0 + i, n1 - 1);
-      a[i] = __ldg(ab + n);
-      x[i] = __ldg(vb + (int64_t)n * 128 + ch);
-    }
+      for (int j = 0; j < 4; ++j) {
+        x0[j] = __ldg(r0 + 32 * j);
+        x1[j] = __ldg(r1 + 32 * j);
+      }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (nb0 + i < n1) {
-        const float v = __uint_as_float((uint32_t)x[i] << 16);
-        acc[a[i] * 128 + ch] += __float2ll_rn(v * 16777216.0f);
-        if (ch == 0) cnt[a[i]] += 1;
+      for (int j = 0; j < 4; ++j) {
+        const int ch = lane + 32 * j;
+        int hi, lo;
+        fix24_split(__uint_as_float((uint32_t)x0[j] << 16), hi, lo);
+        if (hi) atomicAdd(shi + a0 * 128 + ch, hi);
+        atomicAdd(slo + a0 * 128 + ch, lo);
+        if (hb) {
+          fix24_split(__uint_as_float((uint32_t)x1[j] << 16), hi, lo);
+          if (hi) atomicAdd(shi + a1 * 128 + ch, hi);
+          atomicAdd(slo + a1 * 128 + ch, lo);
+        }
+      }
+      if (lane == 0) {
+        atomicAdd(&cnt[a0], 1);
+        if (hb) atomicAdd(&cnt[a1], 1);
       }
     }
+    __syncthreads();
+    for (int i = threadIdx.x; i < k * 128; i += blockDim.x) {
+      tot[i] += ((long long)shi[i] << 22) + (long long)slo[i];
+      shi[i] = 0;
+      slo[i] = 0;
+    }
+    __syncthreads();
   }
-  __syncthreads();
   long long* dst = sums + (int64_t)bh * k * 128;
-  for (int c = 0; c < k; ++c) {
-    long long s = acc[c * 128 + ch];
-    if (s != 0) atomicAdd(reinterpret_cast<unsigned long long*>(dst + c * 128 + ch), (unsigned long long)s);
+  for (int i = threadIdx.x; i < k * 128; i += blockDim.x) {
+    const long long s = tot[i];
+    if (s != 0) atomicAdd(reinterpret_cast<unsigned long long*>(dst + i), (unsigned long long)s);
   }
-  if (ch < k && cnt[ch] != 0) atomicAdd(counts + (int64_t)bh * k + ch, cnt[ch]);
+  if (threadIdx.x < k && cnt[threadIdx.x] != 0) atomicAdd(counts + (int64_t)bh * k + threadIdx.x, cnt[threadIdx.x]);
 }
 
 __global__ void km_update_kernel(const long long* __restrict__ sums, const int* __restrict__ counts,
@@ -271,22 +353,25 @@ static int cluster_permute_impl(const vca_bf16* V, int B, int H, int N, int d, i
   km_init_kernel<<<dim3(BH, k), 128, 0, s>>>(V, init, cent, N, k);
   int rc = check_launch("km_init_kernel");
   if (rc) return rc;
-  const size_t assign_smem = (size_t)((k + 1) / 2) * 128 * sizeof(float2);
-  const size_t accum_smem = (size_t)k * 128 * sizeof(long long);
-  if (cudaFuncSetAttribute(km_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)assign_smem) !=
+  // centroid table padded to 16 or 32 pairs (pads sit at infinity)
+  const int np = (k + 1) / 2 <= 16 ? 16 : 32;
+  const size_t assign_smem = (size_t)np * 128 * sizeof(float2);
+  const size_t accum_smem = (size_t)k * 128 * (sizeof(long long) + 2 * sizeof(int));
+  auto assign_kernel = np == 16 ? km_assign_kernel<16> : km_assign_kernel<32>;
+  if (cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)assign_smem) !=
           cudaSuccess ||
       cudaFuncSetAttribute(km_accum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)accum_smem) !=
           cudaSuccess)
     return fail(VCA_ERR_CUDA, "vca_cluster_permute: cannot set shared-memory size");
-  const dim3 g_assign((N + kAssignThreads - 1) / kAssignThreads, BH);
+  const dim3 g_assign((N + 2 * kAssignThreads - 1) / (2 * kAssignThreads), BH);
   const dim3 g_accum((N + kAccumChunk - 1) / kAccumChunk, BH);
   for (int it = 0; it < iters; ++it) {
-    km_assign_kernel<<<g_assign, kAssignThreads, assign_smem, s>>>(V, cent, assign, N, k);
+    assign_kernel<<<g_assign, kAssignThreads, assign_smem, s>>>(V, cent, assign, N, k);
     if ((rc = check_launch("km_assign_kernel"))) return rc;
     if (cudaMemsetAsync(w.sums, 0, sums_bytes, s) != cudaSuccess ||
         cudaMemsetAsync(w.counts, 0, counts_bytes, s) != cudaSuccess)
       return fail(VCA_ERR_CUDA, "vca_cluster_permute: memset failed");
-    km_accum_kernel<<<g_accum, 128, accum_smem, s>>>(V, assign, w.sums, w.counts, N, k);
+    km_accum_kernel<<<g_accum, kAccumWarps * 32, accum_smem, s>>>(V, assign, w.sums, w.counts, N, k);
     if ((rc = check_launch("km_accum_kernel"))) return rc;
     km_update_kernel<<<dim3(BH, k), 128, 0, s>>>(w.sums, w.counts, cent, k);
     if ((rc = check_launch("km_update_kernel"))) return rc;
