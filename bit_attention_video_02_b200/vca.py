@@ -32,7 +32,7 @@ EXPORTED = [
     "vca_cluster_permute_workspace_size", "vca_cluster_permute", "vca_cluster_permute_noalloc",
     "vca_smooth_quantize_workspace_size", "vca_smooth_quantize_qkv",
     "vca_attention_workspace_size", "vca_attention_fwd",
-    "vca_bf16_attention_workspace_size", "vca_bf16_attention_fwd",
+    "vca_bf16_attention_workspace_size", "vca_bf16_attention_fwd", "vca_schedule_regroup",
 ]
 
 
@@ -70,10 +70,11 @@ def lib() -> ctypes.CDLL:
         L.vca_bf16_attention_workspace_size.restype = sz
         L.vca_bf16_attention_workspace_size.argtypes = [i32, i32, i32]
         L.vca_bf16_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+        L.vca_schedule_regroup.argtypes = [i32, i32, i32, f32]
         for fn in ("vca_reset_status", "vca_check_status", "vca_debug_wait_timeout", "vca_expcast_ref",
                    "vca_e4m3_encode", "vca_cluster_permute", "vca_cluster_permute_noalloc",
                    "vca_smooth_quantize_qkv",
-                   "vca_attention_fwd", "vca_bf16_attention_fwd"):
+                   "vca_attention_fwd", "vca_bf16_attention_fwd", "vca_schedule_regroup"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -244,3 +245,37 @@ def vc_attention(Q, K, V, k: int = 32, iters: int = 3, softmax_scale=None, perm=
         _, _, perm = cluster_permute(V, k, iters, ws=ws, stream=stream)
     ops = smooth_quantize(Q, K, V, perm, ws=ws, stream=stream)
     return attention_fwd(ops, Q.shape[2], softmax_scale, ws=ws, stream=stream)
+
+
+def schedule_regroup(step: int, total_steps: int, reuse: int = 4, group_fraction: float = 0.25) -> bool:
+    """vca_schedule_regroup: does this denoising step regroup (k-means + sort)?"""
+    rc = lib().vca_schedule_regroup(step, total_steps, reuse, group_fraction)
+    if rc < 0:
+        _check(rc)
+    return rc == 1
+
+
+class VCAttentionLayer:
+    """One attention layer across a denoising run: keeps the layer's permutation
+    and centroids between steps, regroups (warm-started from the last
+    centroids) when vca_schedule_regroup says so, quantises and attends every
+    step.  Holds state only; every step of the path runs in the library."""
+
+    def __init__(self, total_steps: int, k: int = 32, iters: int = 3, reuse: int = 4,
+                 group_fraction: float = 0.25, ws: Workspace | None = None):
+        self.total_steps, self.k, self.iters = total_steps, k, iters
+        self.reuse, self.group_fraction = reuse, group_fraction
+        self.ws = ws
+        self.centroids = None
+        self.perm = None
+        self.regrouped_at = []
+
+    def __call__(self, Q, K, V, step: int, softmax_scale=None, stream=None):
+        if self.ws is None:
+            self.ws = Workspace(lib().vca_status_bytes(), V.device)
+        if self.perm is None or schedule_regroup(step, self.total_steps, self.reuse, self.group_fraction):
+            self.centroids, _, self.perm = cluster_permute(V, self.k, self.iters, init=self.centroids,
+                                                           ws=self.ws, stream=stream)
+            self.regrouped_at.append(step)
+        ops = smooth_quantize(Q, K, V, self.perm, ws=self.ws, stream=stream)
+        return attention_fwd(ops, Q.shape[2], softmax_scale, ws=self.ws, stream=stream)

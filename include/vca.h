@@ -143,6 +143,21 @@ int vca_cluster_permute_noalloc(const vca_bf16* V, int B, int H, int N, int d, i
                                 const float* init_centroids, float* centroids, int32_t* assign,
                                 int32_t* perm, vca_stream_t stream);
 
+/* Denoising-schedule reuse of the grouping ([VCA-mtp], abstract and section
+ * "V-Smooth 與 ExpCast-FP8": grouping runs only in the first 25 % of the
+ * denoising steps and each permutation is reused across 4 adjacent steps, which
+ * amortises the grouping to 3-4 % of attention time).  Host function, no GPU
+ * work: returns 1 when step `step` (0-based) of a `total_steps`-step run should
+ * regroup -- call vca_cluster_permute, warm-started from the centroids of the
+ * previous grouping -- and 0 when it should keep the last permutation;
+ * VCA_ERR_INVALID for step < 0, total_steps < 1, step >= total_steps,
+ * reuse < 1 or group_fraction outside (0, 1].
+ * Reading of the pages: a step regroups iff it is step 0, or
+ * step < group_fraction * total_steps and step is a multiple of `reuse`
+ * (defaults 0.25 and 4).  Quantisation (vca_smooth_quantize_qkv) runs at every
+ * step, since Q, K and V change every step. */
+int vca_schedule_regroup(int step, int total_steps, int reuse, float group_fraction);
+
 size_t vca_smooth_quantize_workspace_size(int B, int H, int N);
 
 /* V-Smooth quantisation ([VCA-news] V-Smooth bullet; [VCA-ru] "Решение": the
