@@ -71,6 +71,8 @@ def _declare(L):
     L.vo_smooth_quantize_head.argtypes = [vp] * 4 + [i32, i32] + [vp] * 7
     L.vo_attention_head.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, vp, vp, vp]
     L.vo_attention_head_bf16.argtypes = [vp] * 4 + [i32, i32, f64, vp, i32, i32, vp]
+    L.vo_attention_head_skip.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, f64, vp, vp, vp]
+    L.vo_attention_head_bf16_skip.argtypes = [vp] * 4 + [i32, i32, f64, vp, i32, i32, f64, vp]
     L.vo_exact_attention_head.argtypes = [vp] * 3 + [i32, i32, f64, vp, i32, vp]
     L.vo_num_threads.restype = i32
 
@@ -181,9 +183,10 @@ def _rows(rows, N):
 
 
 def attention_head(ops: dict, N: int, softmax_scale: float, rows=None, flags: int = 0,
-                   want_lblk: bool = False):
+                   want_lblk: bool = False, skip_lambda: float = 0.0):
     """Same-algorithm attention from quantised operands (dict as returned by
-    ``smooth_quantize_head``).  Returns (O [nrows, d] fp64, lse [nrows], lblk)."""
+    ``smooth_quantize_head``).  Returns (O [nrows, d] fp64, lse [nrows], lblk).
+    skip_lambda > 0 applies the Skip Softmax block rejection."""
     rows = _rows(rows, N)
     d = ops["Qq"].shape[1]
     nb = ops["q_scale"].shape[0]
@@ -191,21 +194,21 @@ def attention_head(ops: dict, N: int, softmax_scale: float, rows=None, flags: in
     lse = np.empty(rows.shape[0], np.float64)
     lblk = np.empty((rows.shape[0], nb), np.float64) if want_lblk else None
     c = {k: np.ascontiguousarray(v) for k, v in ops.items()}
-    lib().vo_attention_head(
+    lib().vo_attention_head_skip(
         _p(c["Qq"]), _p(c["q_scale"]), _p(c["Kq"]), _p(c["k_scale"]), _p(c["VrT"]),
         _p(c["v_exp"]), _p(c["v_mean"]), N, d, float(softmax_scale), _p(rows),
-        rows.shape[0], int(flags), _p(O), _p(lse), _p(lblk) if lblk is not None else None)
+        rows.shape[0], int(flags), float(skip_lambda), _p(O), _p(lse), _p(lblk) if lblk is not None else None)
     return O, lse, lblk
 
 
-def attention_head_bf16(Q, K, V, perm, softmax_scale: float, rows=None, flags: int = 0):
+def attention_head_bf16(Q, K, V, perm, softmax_scale: float, rows=None, flags: int = 0, skip_lambda: float = 0.0):
     Q, K, V = (np.ascontiguousarray(a, dtype=np.uint16) for a in (Q, K, V))
     perm = np.ascontiguousarray(perm, dtype=np.int32)
     N, d = Q.shape
     rows = _rows(rows, N)
     O = np.empty((rows.shape[0], d), np.float64)
-    lib().vo_attention_head_bf16(_p(Q), _p(K), _p(V), _p(perm), N, d, float(softmax_scale),
-                                 _p(rows), rows.shape[0], int(flags), _p(O))
+    lib().vo_attention_head_bf16_skip(_p(Q), _p(K), _p(V), _p(perm), N, d, float(softmax_scale),
+                                      _p(rows), rows.shape[0], int(flags), float(skip_lambda), _p(O))
     return O
 
 

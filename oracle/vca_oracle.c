@@ -359,7 +359,7 @@ void vo_smooth_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_
  * every code <= 56 + 8*(VO_HEADROOM + VO_LAG) = 120 < 126. */
 static void attn_row(const double* q, double qs, const double* kh, const double* ks,
                      const double* rh, const int* vexp, const double* mu, int N, int d,
-                     double softmax_scale, int flags, double* O, double* lse,
+                     double softmax_scale, int flags, double skip_log2, double* O, double* lse,
                      double* lblk, double* z /* scratch [N] */, double* acc /* [d] */) {
     const double log2e = 1.4426950408889634074;
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
@@ -369,12 +369,23 @@ static void attn_row(const double* q, double qs, const double* kh, const double*
         z[j] = s * qs * ks[j] * softmax_scale * log2e;
     }
     for (int c = 0; c < d; ++c) acc[c] = 0.0;
-    double ltot = 0.0, n = 0.0;
+    double ltot = 0.0, n = 0.0, zrun = -INFINITY;
     for (int b = 0; b < nb; ++b) {
         int j0 = b * VO_BLOCK, j1 = j0 + VO_BLOCK < N ? j0 + VO_BLOCK : N;
         double zmax = -INFINITY;
         for (int j = j0; j < j1; ++j)
             if (z[j] > zmax) zmax = z[j];
+        /* Skip Softmax (BLASST): the block is negligible for this row when
+         * exp(block max - running max) < lambda, i.e. in log2 units
+         * zmax - zrun < log2(lambda); it then adds nothing (no probabilities,
+         * no PV, zero row sum).  skip_log2 = -inf disables the rule.  A
+         * rejected block lies below the running maximum, which the reference
+         * trails by at most VO_LAG octaves, so it could not move the reference. */
+        if (zmax > zrun) zrun = zmax;
+        if (b > 0 && zmax - zrun < skip_log2) {
+            if (lblk) lblk[b] = 0.0;
+            continue;
+        }
         double nblk = ceil(zmax - VO_PHI);
         if (b == 0) {
             n = nblk;
@@ -420,7 +431,7 @@ static void attn_row(const double* q, double qs, const double* kh, const double*
 static void attn_rows(const double* qh, const double* qs_row, const double* kh,
                       const double* ks, const double* rh, const int* vexp,
                       const double* mu, int N, int d, double softmax_scale,
-                      const int32_t* rows, int nrows, int flags, double* O,
+                      const int32_t* rows, int nrows, int flags, double skip_log2, double* O,
                       double* lse, double* lblk) {
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
 #pragma omp parallel
@@ -431,7 +442,7 @@ static void attn_rows(const double* qh, const double* qs_row, const double* kh,
         for (int r = 0; r < nrows; ++r) {
             int i = rows[r];
             attn_row(qh + (int64_t)i * d, qs_row[i], kh, ks, rh, vexp, mu, N, d,
-                     softmax_scale, flags, O + (int64_t)r * d, lse ? &lse[r] : NULL,
+                     softmax_scale, flags, skip_log2, O + (int64_t)r * d, lse ? &lse[r] : NULL,
                      lblk ? lblk + (int64_t)r * nb : NULL, z, acc);
         }
         free(z);
@@ -439,11 +450,22 @@ static void attn_rows(const double* qh, const double* qs_row, const double* kh,
     }
 }
 
+static double skip_log2_of(double lambda) { return lambda > 0.0 ? log2(lambda) : -INFINITY; }
+
 void vo_attention_head(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
                        const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
                        const uint16_t* v_mean, int N, int d, double softmax_scale,
                        const int32_t* rows, int nrows, int flags,
                        double* O, double* lse, double* lblk) {
+    vo_attention_head_skip(Qq, q_scale, Kq, k_scale, VrT, v_exp, v_mean, N, d, softmax_scale, rows, nrows,
+                           flags, 0.0, O, lse, lblk);
+}
+
+void vo_attention_head_skip(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                            const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                            const uint16_t* v_mean, int N, int d, double softmax_scale,
+                            const int32_t* rows, int nrows, int flags, double skip_lambda,
+                            double* O, double* lse, double* lblk) {
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
     int64_t Np = (int64_t)nb * VO_BLOCK;
     double* qh = (double*)malloc((size_t)N * d * sizeof(double));
@@ -466,13 +488,20 @@ void vo_attention_head(const uint8_t* Qq, const float* q_scale, const uint8_t* K
         ve[b] = v_exp[b];
         for (int c = 0; c < d; ++c) mu[(int64_t)b * d + c] = vo_bf16_to_float(v_mean[(int64_t)b * d + c]);
     }
-    attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, O, lse, lblk);
+    attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, skip_log2_of(skip_lambda), O,
+              lse, lblk);
     free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
 }
 
 void vo_attention_head_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                             const int32_t* perm, int N, int d, double softmax_scale,
                             const int32_t* rows, int nrows, int flags, double* O) {
+    vo_attention_head_bf16_skip(Q, K, V, perm, N, d, softmax_scale, rows, nrows, flags, 0.0, O);
+}
+
+void vo_attention_head_bf16_skip(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                 const int32_t* perm, int N, int d, double softmax_scale,
+                                 const int32_t* rows, int nrows, int flags, double skip_lambda, double* O) {
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
     int64_t Np = (int64_t)nb * VO_BLOCK;
     if (!(flags & VO_IDENTITY_QUANT)) {
@@ -484,8 +513,8 @@ void vo_attention_head_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t
         int8_t* ve = (int8_t*)malloc((size_t)nb);
         uint16_t* vm = (uint16_t*)malloc((size_t)nb * d * sizeof(uint16_t));
         vo_smooth_quantize_head(Q, K, V, perm, N, d, Qq, qsc, Kq, ksc, VrT, ve, vm);
-        vo_attention_head(Qq, qsc, Kq, ksc, VrT, ve, vm, N, d, softmax_scale, rows, nrows,
-                          flags, O, NULL, NULL);
+        vo_attention_head_skip(Qq, qsc, Kq, ksc, VrT, ve, vm, N, d, softmax_scale, rows, nrows,
+                               flags, skip_lambda, O, NULL, NULL);
         free(Qq); free(Kq); free(VrT); free(qsc); free(ksc); free(ve); free(vm);
         return;
     }
@@ -514,8 +543,8 @@ void vo_attention_head_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t
             for (int j = j0; j < j1; ++j) rh[(int64_t)j * d + c] -= m;
         }
     }
-    attn_rows(qh, ones, kh, ones, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, O,
-              NULL, NULL);
+    attn_rows(qh, ones, kh, ones, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags,
+              skip_log2_of(skip_lambda), O, NULL, NULL);
     free(qh); free(kh); free(rh); free(ones); free(mu); free(ve);
 }
 

@@ -84,11 +84,26 @@ void vo_attention_head(const uint8_t* Qq, const float* q_scale, const uint8_t* K
                        const int32_t* rows, int nrows, int flags,
                        double* O, double* lse, double* lblk);
 
+/* Same, with Skip Softmax (BLASST, "Accelerating Video Generation with GEMM
+ * Quantization, Attention Quantization and Skip Softmax Attention in
+ * TensorRT-LLM", section "Sparse Attention with Skip Softmax"): key block j is
+ * dropped for row i when exp(block max - running max) < skip_lambda (scores in
+ * natural-log units; the running max includes block j).  skip_lambda = 0 is
+ * the plain algorithm; 0 <= skip_lambda < 1. */
+void vo_attention_head_skip(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                            const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                            const uint16_t* v_mean, int N, int d, double softmax_scale,
+                            const int32_t* rows, int nrows, int flags, double skip_lambda,
+                            double* O, double* lse, double* lblk);
+
 /* Same algorithm, straight from bf16 Q/K/V and a permutation; with
  * VO_IDENTITY_QUANT the quantisers are the identity (for reductions). */
 void vo_attention_head_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
                             const int32_t* perm, int N, int d, double softmax_scale,
                             const int32_t* rows, int nrows, int flags, double* O);
+void vo_attention_head_bf16_skip(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                 const int32_t* perm, int N, int d, double softmax_scale,
+                                 const int32_t* rows, int nrows, int flags, double skip_lambda, double* O);
 
 /* Exact fp64 softmax(Q K^T * scale) V for selected rows of one head. */
 void vo_exact_attention_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V,

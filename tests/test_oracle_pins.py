@@ -451,3 +451,75 @@ def test_same_algorithm_invariant_to_key_order_within_rounding():
     ex = oracle.exact_attention_head(Q, K, V, sc)
     for o in (a, c):
         assert np.linalg.norm(o - ex) / np.linalg.norm(ex) < 0.08
+
+
+# ------------------------------------------------------------------ Skip Softmax (BLASST)
+def _skip_case(seed=31, N=700):
+    # strong and weak key blocks alternate: the weak ones sit ~6 natural-log
+    # units below the running maximum (rejected at lambda = 2^-6), the strong
+    # ones within ~1 unit of it (kept)
+    rng = np.random.default_rng(seed)
+    qf = np.abs(rng.standard_normal((N, 128))) * 0.4
+    kf = np.abs(rng.standard_normal((N, 128))) * 0.2
+    blk = np.arange(N) // 128
+    factor = np.array([12.0, 1.0, 11.5, 1.5, 12.0, 0.5, 11.0, 1.0])
+    kf *= factor[blk % len(factor)][:, None]
+    return bf16_bits_of(qf), bf16_bits_of(kf), _bits(rng, N)
+
+
+def _survivors(Q, K, sc, lam, rows):
+    # rejection decided from fp64 logits: block max vs the running max (which
+    # includes the block), natural-log units
+    q = bits_to_f32(Q).astype(np.float64)[rows]
+    k = bits_to_f32(K).astype(np.float64)
+    s = q @ k.T * sc
+    N = k.shape[0]
+    keep = np.ones_like(s, dtype=bool)
+    for r in range(len(rows)):
+        run = -np.inf
+        for b in range(0, N, 128):
+            m = s[r, b:b + 128].max()
+            run = max(run, m)
+            if b > 0 and np.exp(m - run) < lam:
+                keep[r, b:b + 128] = False
+    return keep
+
+
+def test_skip_softmax_equals_exact_attention_over_the_kept_blocks():
+    Q, K, V = _skip_case()
+    N = Q.shape[0]
+    perm = np.arange(N, dtype=np.int32)
+    sc = 1 / math.sqrt(128)
+    rows = np.arange(0, N, 23, dtype=np.int32)
+    lam = 2.0 ** -6
+    keep = _survivors(Q, K, sc, lam, rows)
+    assert 0.05 < 1 - keep.mean() < 0.95           # the case really rejects blocks, not all
+    fl = oracle.EXACT_EXP | oracle.IDENTITY_QUANT
+    got = oracle.attention_head_bf16(Q, K, V, perm, sc, rows=rows, flags=fl, skip_lambda=lam)
+    vf = bits_to_f32(V).astype(np.float64)
+    q = bits_to_f32(Q).astype(np.float64)[rows]
+    k = bits_to_f32(K).astype(np.float64)
+    s = q @ k.T * sc
+    for r in range(len(rows)):
+        kk = keep[r]
+        p = np.exp(s[r, kk] - s[r, kk].max())
+        want = p @ vf[kk] / p.sum()
+        assert np.abs(got[r] - want).max() < 1e-10
+    # without the rule it is plain exact attention, which differs
+    full = oracle.attention_head_bf16(Q, K, V, perm, sc, rows=rows, flags=fl)
+    assert np.abs(full - got).max() > 1e-6
+
+
+def test_skip_softmax_zero_lambda_is_the_plain_algorithm():
+    Q, K, V = _skip_case(seed=32, N=400)
+    perm = np.arange(Q.shape[0], dtype=np.int32)
+    ops = oracle.smooth_quantize_head(Q, K, V, perm)
+    a, la, _ = oracle.attention_head(ops, Q.shape[0], 1 / math.sqrt(128))
+    b, lb, _ = oracle.attention_head(ops, Q.shape[0], 1 / math.sqrt(128), skip_lambda=0.0)
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+    # rejected blocks contribute a zero row sum
+    rows = np.arange(0, Q.shape[0], 9, dtype=np.int32)
+    _, _, lblk = oracle.attention_head(ops, Q.shape[0], 1 / math.sqrt(128), rows=rows, want_lblk=True,
+                                       skip_lambda=2.0 ** -6)
+    keep = _survivors(Q, K, 1 / math.sqrt(128), 2.0 ** -6, rows)[:, ::128]
+    assert np.all(lblk[~keep] == 0.0) and np.all(lblk[keep] > 0.0)
