@@ -64,7 +64,22 @@ struct AttnParams {
   float c_base;            // softmax_scale * log2(e)
   DevStatus* st;
   unsigned long long wait_ns;
+  float skip_log2;               // Skip Softmax: log2(lambda), -inf when off
+  unsigned long long* skipped;   // optional count of skipped (query tile, key block) pairs
 };
+
+// AND of a predicate over the 128 threads of one softmax warpgroup (named
+// barrier `id`); every thread of the warpgroup must reach it.
+__device__ __forceinline__ bool wg_and(bool v, int id) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v), "r"(id)
+      : "memory");
+  return out != 0;
+}
 
 struct __align__(8) AttnBars {
   uint64_t q_full;
@@ -83,6 +98,13 @@ __device__ __forceinline__ uint32_t tf32_tile_off(int r, int k) {
   return (uint32_t)((r >> 3) * 256 + (k >> 2) * 128 + (r & 7) * 16 + (k & 3) * 4);
 }
 
+// SKIP: Skip Softmax (BLASST) block rejection ("Accelerating Video Generation
+// with GEMM Quantization, Attention Quantization and Skip Softmax Attention in
+// TensorRT-LLM", section "Sparse Attention with Skip Softmax"): row i drops key
+// block j when exp(block max - running max) < lambda.  Rejected rows write code
+// 0 (no probability, zero row sum); when all 128 rows of a query tile reject a
+// block, the tile skips its code pass and the MMA warp skips its PV.
+template <bool SKIP>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -90,6 +112,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int never_s;   // abort flag for drain waits: these must not give up early
+  __shared__ int pv_skip_s[2];   // Skip Softmax: the current PV of tile t is skipped
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
@@ -101,6 +124,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
   if (threadIdx.x == 0) {
     abort_s = 0;
     never_s = 0;
+    pv_skip_s[0] = pv_skip_s[1] = 0;
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars.kv_full[s], 1);
@@ -195,10 +219,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         if (!ok) break;
         tc_fence_after();
         const uint32_t sft = tmem + t * 128;   // scale vectors live in the consumed S_t columns
+        // (the flag was written before the warpgroup's p_full arrivals)
+        const bool skip_pv = SKIP && *reinterpret_cast<volatile int*>(&pv_skip_s[t]) != 0;
+        if (!skip_pv) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k)   // P_t at S_t columns 8..39, 8 columns (32 codes) per K step
-          mma_mxf8_ts_w(tmem + 256 + t * 128, sft + 8 + 8 * k, dV + (uint64_t)(s * 1024 + 2 * k), id_pv, sft,
-                        sft + 4, (j > 0 || k > 0) ? 1u : 0u);
+          for (int k = 0; k < 4; ++k)   // P_t at S_t columns 8..39, 8 columns (32 codes) per K step
+            mma_mxf8_ts_w(tmem + 256 + t * 128, sft + 8 + 8 * k, dV + (uint64_t)(s * 1024 + 2 * k), id_pv, sft,
+                          sft + 4, (j > 0 || k > 0) ? 1u : 0u);
+        }
         if (group_end) {
           ok = mbar_wait_warp(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220);
           if (!ok) break;
@@ -253,6 +281,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const uint32_t tO = tmem + 256 + t * 128 + lane_off;
     const int qtile = pair * 2 + t;
     const bool qvalid = qtile < nb;
+    const bool row_valid = qvalid && qtile * 128 + r < N;
     const float sq = qvalid ? __ldg(p.q_scale + (int64_t)bh * nb + qtile) : 1.0f;
     const float cq = sq * p.c_base;
     const float kMagic = 12582912.0f;              // 1.5 * 2^23: adding it rounds to an integer
@@ -261,6 +290,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const int8_t* vex = p.v_exp + (int64_t)bh * nb;
     int nref = 0;
     bool have_ref = false;
+    float zrun = -INFINITY;        // Skip Softmax: running maximum of the block maxima (log2 units)
+    unsigned long long nskip = 0;
     float ltot = 0.0f;
     bool ok = true;
     // the next tile's K scale and V exponent are loaded one tile ahead, off the
@@ -275,6 +306,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         vex_next = __ldg(vex + j + 1);
       }
       ok = mbar_wait_warp(&bars.s_full[t], j & 1, &abort_s, p.st, lim, 400 + t);
+      // with SKIP the warpgroup votes below through named barriers, so its four
+      // warps must leave the loop together
+      if (SKIP) ok = wg_and(ok, 1 + t);
       if (!ok) break;
       tc_fence_after();
       float sv[128];
@@ -305,11 +339,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
       const float cz = cq * ksc_j;                 // z = s * cz (log2 domain)
       const float c8 = 8.0f * cz;
+      bool rej = false;           // Skip Softmax: this row drops the block
+      if (SKIP) {
+        const float zt = mx * cz;
+        zrun = fmaxf(zrun, zt);
+        // rows past the end of the sequence (padding of the last query tile)
+        // vote to drop every block, so they never hold a whole-tile skip back
+        rej = j > 0 && (!row_valid || zt - zrun < p.skip_log2);
+      }
       const int ntile = (int)ceilf(__fmaf_rn(mx, cz, -0.08125f));
       // (S_t(j) was committed after PV_t(j-1) and any mean MMA before it, so
       // those have completed: O_t may be rescaled and sL_t rewritten now)
       float rescale = 1.0f;       // O_t and the pending row sums are scaled by this
-      if (!have_ref) {
+      if (rej) {
+        // a dropped block lies below the running maximum, which the reference
+        // trails by at most 4 octaves: it leaves the reference where it is
+      } else if (!have_ref) {
         nref = ntile;
         have_ref = true;
       } else if (ntile > nref + 4) {
@@ -320,10 +365,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       // ExpCast: code = rne(s*c8 + 87 - 8*nref) via the magic-number FMA (two
       // scores per fma.rn.f32x2), clamped below at 0; the decoded probability is
       // float(code << 20) * 2^120, summed exactly enough in fp32 pairs
-      const float badd = kMagic + (float)(87 - 8 * nref);
-      const float2 c8x2 = make_float2(c8, c8), baddx2 = make_float2(badd, badd);
+      const bool tile_skip = SKIP && wg_and(rej, 1 + t);
+      // a dropped row writes code 0 everywhere: multiplier 0, addend the bare magic constant
+      const float badd = rej ? kMagic : kMagic + (float)(87 - 8 * nref);
+      const float c8r = rej ? 0.0f : c8;
+      const float2 c8x2 = make_float2(c8r, c8r), baddx2 = make_float2(badd, badd);
       float2 lsa = make_float2(0.0f, 0.0f), lsb = make_float2(0.0f, 0.0f);
       uint32_t pw[32];   // the row's 128 codes, 4 per word, in key order
+      if (!tile_skip) {
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
         const int c = q * 4;
@@ -336,6 +385,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         pw[q] = prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
       }
       VCA_TMEM_ST32(tS + 8, pw);
+      }
       const float lsum = (lsa.x + lsa.y) + (lsb.x + lsb.y);
       const float l = lsum * 0x1p120f;
       // block row sum -> L tile (hi part exact in TF32, lo the remainder)
@@ -374,7 +424,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       }
       ltot = ltot * rescale + l;
       // UE8M0 scale vectors for this PV: A = 2^0, B = 2^v_exp[j]
-      {
+      if (!tile_skip) {
         const uint32_t eb = (uint32_t)(127 + vex_j);
         uint32_t sf[8];
 #pragma unroll
@@ -383,11 +433,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         for (int i = 4; i < 8; ++i) sf[i] = eb * 0x01010101u;
         tmem_st8(tS, sf);
       }
+      if (SKIP && r == 0) {
+        pv_skip_s[t] = tile_skip ? 1 : 0;
+        nskip += tile_skip ? 1 : 0;
+      }
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars.p_full[t]);
     }
+    if (SKIP && r == 0 && p.skipped && nskip) atomicAdd(p.skipped, nskip);
     // ------------------------------------------------------------ epilogue
     if (ok) ok = mbar_wait_warp(&bars.o_done[t], (nkv - 1) & 1, &abort_s, p.st, lim, 420 + t);
     if (ok) {
@@ -436,27 +491,29 @@ using namespace vca;
 
 extern "C" size_t vca_attention_workspace_size(int B, int H, int N) { return 256; }
 
-extern "C" int vca_attention_fwd(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
-                                 const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
-                                 const vca_bf16* v_mean, int B, int H, int N, int d,
-                                 float softmax_scale, vca_bf16* O, float* lse, void* ws,
-                                 size_t ws_bytes, vca_stream_t stream) {
-  if (d != VCA_HEAD_DIM) return fail(VCA_ERR_UNSUPPORTED, "vca_attention_fwd: d must be 128");
+static int attention_launch(const char* fn, const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                            const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                            const vca_bf16* v_mean, int B, int H, int N, int d, float softmax_scale,
+                            vca_bf16* O, float* lse, void* ws, size_t ws_bytes, float skip_lambda,
+                            unsigned long long* skipped, vca_stream_t stream) {
+  if (d != VCA_HEAD_DIM) return fail(VCA_ERR_UNSUPPORTED, "%s: d must be 128", fn);
   if (B < 1 || H < 1 || N < 1 || (int64_t)B * H > 65535)
-    return fail(VCA_ERR_INVALID, "vca_attention_fwd: bad shape B=%d H=%d N=%d", B, H, N);
+    return fail(VCA_ERR_INVALID, "%s: bad shape B=%d H=%d N=%d", fn, B, H, N);
   const int nb = (N + 127) / 128;
   const int64_t Np = (int64_t)nb * 128;
   if ((int64_t)B * H * Np > INT32_MAX || Np > INT32_MAX / 2)
-    return fail(VCA_ERR_UNSUPPORTED, "vca_attention_fwd: B*H*Np exceeds the 2^31 row limit");
+    return fail(VCA_ERR_UNSUPPORTED, "%s: B*H*Np exceeds the 2^31 row limit", fn);
   const void* ptrs[] = {Qq, q_scale, Kq, k_scale, VrT, v_exp, v_mean, O};
   for (const void* q : ptrs)
-    if (!q) return fail(VCA_ERR_INVALID, "vca_attention_fwd: null pointer");
+    if (!q) return fail(VCA_ERR_INVALID, "%s: null pointer", fn);
   const void* al[] = {Qq, Kq, VrT, O};
   for (const void* q : al)
-    if (!aligned16(q)) return fail(VCA_ERR_INVALID, "vca_attention_fwd: tensors must be 16-byte aligned");
-  if (!(softmax_scale > 0.0f)) return fail(VCA_ERR_INVALID, "vca_attention_fwd: softmax_scale must be > 0");
+    if (!aligned16(q)) return fail(VCA_ERR_INVALID, "%s: tensors must be 16-byte aligned", fn);
+  if (!(softmax_scale > 0.0f)) return fail(VCA_ERR_INVALID, "%s: softmax_scale must be > 0", fn);
+  if (!(skip_lambda >= 0.0f && skip_lambda < 1.0f))
+    return fail(VCA_ERR_INVALID, "%s: skip_lambda must be in [0, 1)", fn);
   if (!ws || ws_bytes < vca_attention_workspace_size(B, H, N))
-    return fail(VCA_ERR_WORKSPACE, "vca_attention_fwd: workspace too small");
+    return fail(VCA_ERR_WORKSPACE, "%s: workspace too small", fn);
 
   AttnParams prm;
   const uint64_t BH = (uint64_t)B * H;
@@ -480,10 +537,32 @@ extern "C" int vca_attention_fwd(const uint8_t* Qq, const float* q_scale, const 
   prm.c_base = (float)((double)softmax_scale * 1.4426950408889634);
   prm.st = (DevStatus*)ws;
   prm.wait_ns = wait_limit_ns();
-  if (cudaFuncSetAttribute(attn_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc) !=
-      cudaSuccess)
-    return fail(VCA_ERR_CUDA, "vca_attention_fwd: cannot set shared-memory size");
+  const bool skip = skip_lambda > 0.0f;
+  prm.skip_log2 = skip ? (float)log2((double)skip_lambda) : -INFINITY;
+  prm.skipped = skipped;
+  auto kern = skip ? attn_fp8_kernel<true> : attn_fp8_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc) != cudaSuccess)
+    return fail(VCA_ERR_CUDA, "%s: cannot set shared-memory size", fn);
   dim3 grid((nb + 1) / 2, (unsigned)BH);
-  attn_fp8_kernel<<<grid, kAttnThreads, kSmemAlloc, (cudaStream_t)stream>>>(prm);
+  kern<<<grid, kAttnThreads, kSmemAlloc, (cudaStream_t)stream>>>(prm);
   return check_launch("attn_fp8_kernel");
+}
+
+extern "C" int vca_attention_fwd(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                                 const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                                 const vca_bf16* v_mean, int B, int H, int N, int d,
+                                 float softmax_scale, vca_bf16* O, float* lse, void* ws,
+                                 size_t ws_bytes, vca_stream_t stream) {
+  return attention_launch("vca_attention_fwd", Qq, q_scale, Kq, k_scale, VrT, v_exp, v_mean, B, H, N, d,
+                          softmax_scale, O, lse, ws, ws_bytes, 0.0f, nullptr, stream);
+}
+
+extern "C" int vca_attention_fwd_skip(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                                      const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                                      const vca_bf16* v_mean, int B, int H, int N, int d,
+                                      float softmax_scale, float skip_lambda, vca_bf16* O, float* lse,
+                                      unsigned long long* skipped_tiles, void* ws, size_t ws_bytes,
+                                      vca_stream_t stream) {
+  return attention_launch("vca_attention_fwd_skip", Qq, q_scale, Kq, k_scale, VrT, v_exp, v_mean, B, H, N, d,
+                          softmax_scale, O, lse, ws, ws_bytes, skip_lambda, skipped_tiles, stream);
 }

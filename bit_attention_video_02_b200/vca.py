@@ -33,6 +33,7 @@ EXPORTED = [
     "vca_smooth_quantize_workspace_size", "vca_smooth_quantize_qkv",
     "vca_attention_workspace_size", "vca_attention_fwd",
     "vca_bf16_attention_workspace_size", "vca_bf16_attention_fwd", "vca_schedule_regroup",
+    "vca_attention_fwd_skip",
 ]
 
 
@@ -71,10 +72,12 @@ def lib() -> ctypes.CDLL:
         L.vca_bf16_attention_workspace_size.argtypes = [i32, i32, i32]
         L.vca_bf16_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
         L.vca_schedule_regroup.argtypes = [i32, i32, i32, f32]
+        L.vca_attention_fwd_skip.argtypes = [vp] * 7 + [i32, i32, i32, i32, f32, f32, vp, vp, vp, vp, sz, vp]
         for fn in ("vca_reset_status", "vca_check_status", "vca_debug_wait_timeout", "vca_expcast_ref",
                    "vca_e4m3_encode", "vca_cluster_permute", "vca_cluster_permute_noalloc",
                    "vca_smooth_quantize_qkv",
-                   "vca_attention_fwd", "vca_bf16_attention_fwd", "vca_schedule_regroup"):
+                   "vca_attention_fwd", "vca_bf16_attention_fwd", "vca_schedule_regroup",
+                   "vca_attention_fwd_skip"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -221,6 +224,29 @@ def attention_fwd(ops: dict, N: int, softmax_scale: float | None = None, O=None,
         _ptr(ops["Qq"]), _ptr(ops["q_scale"]), _ptr(ops["Kq"]), _ptr(ops["k_scale"]), _ptr(ops["VrT"]),
         _ptr(ops["v_exp"]), _ptr(ops["v_mean"]), B, H, N, d, scale, _ptr(O), _ptr(lse), ws.ptr, ws.nbytes,
         _stream(stream)))
+    return (O, lse) if want_lse else O
+
+
+def attention_fwd_skip(ops: dict, N: int, skip_lambda: float, softmax_scale: float | None = None, O=None,
+                       lse=None, want_lse: bool = False, skipped=None, ws: Workspace | None = None, stream=None):
+    """vca_attention_fwd_skip: attention with Skip Softmax block rejection.
+    `skipped`, if given, is a one-element int64 device tensor the number of
+    skipped (query tile, key block) pairs is added to."""
+    B, H, Np, d = ops["Qq"].shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dev = ops["Qq"].device
+    if O is None:
+        O = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    if skipped is not None:
+        assert skipped.dtype == torch.int64 and skipped.numel() == 1
+    need = lib().vca_attention_workspace_size(B, H, N)
+    ws = (ws or Workspace(need, dev)).ensure(need)
+    _check(lib().vca_attention_fwd_skip(
+        _ptr(ops["Qq"]), _ptr(ops["q_scale"]), _ptr(ops["Kq"]), _ptr(ops["k_scale"]), _ptr(ops["VrT"]),
+        _ptr(ops["v_exp"]), _ptr(ops["v_mean"]), B, H, N, d, scale, float(skip_lambda), _ptr(O), _ptr(lse),
+        _ptr(skipped), ws.ptr, ws.nbytes, _stream(stream)))
     return (O, lse) if want_lse else O
 
 

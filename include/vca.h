@@ -211,6 +211,27 @@ int vca_attention_fwd(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq
                       const vca_bf16* v_mean, int B, int H, int N, int d, float softmax_scale,
                       vca_bf16* O, float* lse, void* ws, size_t ws_bytes, vca_stream_t stream);
 
+/* Same attention with Skip Softmax (BLASST) block rejection ([TRT-blog],
+ * section "Sparse Attention with Skip Softmax": a score block is dropped for a
+ * query row when exp(block max - running max) < lambda; dropped blocks skip the
+ * exponentiation and their PV accumulation).  Row i drops key block b when
+ *   z~_ib - max_{b' <= b} z~_ib' < log2(skip_lambda),  z~_ib = max_{j in b} z_ij
+ * (z as in vca_attention_fwd, log2 units), except block 0, which is always
+ * kept.  A dropped block adds no probabilities, no PV and a zero row sum; it
+ * never moves the reference n.  When every row of a 128-row query tile drops a
+ * block, the kernel also skips that tile's code pass and PV MMA.
+ *   skip_lambda     in [0, 1); 0 gives exactly vca_attention_fwd
+ *   skipped_tiles   optional device counter (one uint64, not zeroed here): the
+ *                   number of (query tile, key block) pairs skipped is added
+ * Errors as vca_attention_fwd, plus VCA_ERR_INVALID for skip_lambda outside
+ * [0, 1). */
+int vca_attention_fwd_skip(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                           const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                           const vca_bf16* v_mean, int B, int H, int N, int d, float softmax_scale,
+                           float skip_lambda, vca_bf16* O, float* lse,
+                           unsigned long long* skipped_tiles, void* ws, size_t ws_bytes,
+                           vca_stream_t stream);
+
 /* In-repo BF16 comparator: exact-softmax flash attention (online softmax with
  * exp2), tcgen05 BF16 MMAs with fp32 accumulation in tensor memory.
  *   Q, K, V, O [B][H][N][d] bf16; lse [B][H][N] fp32 natural log (nullable). */
