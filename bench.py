@@ -221,6 +221,52 @@ def run_ours(args, world, rank, local):
         bf16_ms = b0.elapsed_time(b1) / 3
     ws.check()
 
+    # ---- Skip Softmax (BLASST) variant: on the workload itself, and on a
+    # block-sparse version of it (K scaled x12 on every other key block, identity
+    # order) where whole query tiles drop the weak blocks
+    skip = None
+    if not args.no_skip:
+        lam = args.skip_lambda
+        nb = (N + 127) // 128
+        pairs = B * H * ((nb + 1) // 2 * 2) * nb
+
+        def time_skip(o, reps=3):
+            cnt = torch.zeros(1, dtype=torch.int64, device=dev)
+            vca.attention_fwd_skip(o, N, lam, O=O, skipped=cnt, ws=ws)
+            torch.cuda.synchronize()
+            cnt.zero_()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(reps):
+                vca.attention_fwd_skip(o, N, lam, O=O, skipped=cnt, ws=ws)
+            s1.record(stream)
+            torch.cuda.synchronize()
+            return s0.elapsed_time(s1) / reps, cnt.item() / reps / pairs
+
+        ms_w, frac_w = time_skip(ops)
+        ident = torch.arange(N, dtype=torch.int32, device=dev).expand(B, H, N).contiguous()
+        blk = torch.arange(N, device=dev) // 128
+        K2 = K * torch.where(blk % 2 == 0, 12.0, 1.0).to(K.dtype)[None, None, :, None]
+        ops2 = vca.alloc_quantized(B, H, N, dev)
+        vca.smooth_quantize(Q, K2, V, ident, out=ops2, ws=ws)
+        del K2
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        vca.attention_fwd(ops2, N, scale, O=O, ws=ws)
+        d0.record(stream)
+        for _ in range(3):
+            vca.attention_fwd(ops2, N, scale, O=O, ws=ws)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = d0.elapsed_time(d1) / 3
+        ms_s, frac_s = time_skip(ops2)
+        del ops2
+        skip = {"lambda": lam,
+                "workload": {"attn_ms": round(ms_w, 3), "skipped_tile_frac": round(frac_w, 4)},
+                "block_sparse_case": {"dense_attn_ms": round(dense_ms, 3), "skip_attn_ms": round(ms_s, 3),
+                                      "skipped_tile_frac": round(frac_s, 4),
+                                      "what": "workload Q, V; K x12 on even key blocks; identity order"}}
+        ws.check()
+
     # ---- end to end through the C ABI with host buffers
     e2e = None
     if not args.no_e2e:
@@ -291,6 +337,7 @@ def run_ours(args, world, rank, local):
         "prep_ms": round(prep_ms, 3),
         "quant_only_ms": round(quant_ms, 3),
         "bf16_attn_ms": round(bf16_ms, 3) if bf16_ms else None,
+        "skip_softmax": skip,
         "fp8_over_bf16": round(bf16_ms / (t_attn * 1e3), 3) if bf16_ms else None,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp8_peak_sust, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / fp8_peak_sust, 4), "traffic": traffic,
@@ -426,6 +473,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bf16", action="store_true")
+    ap.add_argument("--no-skip", action="store_true")
+    ap.add_argument("--skip-lambda", type=float, default=2.0 ** -6)
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
     if args.gpus != world and rank == 0:
