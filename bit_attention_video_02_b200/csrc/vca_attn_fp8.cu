@@ -68,18 +68,6 @@ struct AttnParams {
   unsigned long long* skipped;   // optional count of skipped (query tile, key block) pairs
 };
 
-// AND of a predicate over the 128 threads of one softmax warpgroup (named
-// barrier `id`); every thread of the warpgroup must reach it.
-__device__ __forceinline__ bool wg_and(bool v, int id) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(out)
-      : "r"((uint32_t)v), "r"(id)
-      : "memory");
-  return out != 0;
-}
 
 struct __align__(8) AttnBars {
   uint64_t q_full;
@@ -102,8 +90,9 @@ __device__ __forceinline__ uint32_t tf32_tile_off(int r, int k) {
 // with GEMM Quantization, Attention Quantization and Skip Softmax Attention in
 // TensorRT-LLM", section "Sparse Attention with Skip Softmax"): row i drops key
 // block j when exp(block max - running max) < lambda.  Rejected rows write code
-// 0 (no probability, zero row sum); when all 128 rows of a query tile reject a
-// block, the tile skips its code pass and the MMA warp skips its PV.
+// 0 (no probability, zero row sum); a warp whose 32 rows all reject skips its
+// code pass (it stores zero codes), and when all four warps of a query tile do,
+// the MMA warp skips the tile's PV.
 template <bool SKIP>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -112,7 +101,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int never_s;   // abort flag for drain waits: these must not give up early
-  __shared__ int pv_skip_s[2];   // Skip Softmax: the current PV of tile t is skipped
+  __shared__ int warp_drop_s[2][4];   // Skip Softmax: warp w of tile t dropped the current block
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
@@ -124,7 +113,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
   if (threadIdx.x == 0) {
     abort_s = 0;
     never_s = 0;
-    pv_skip_s[0] = pv_skip_s[1] = 0;
+    for (int i = 0; i < 8; ++i) warp_drop_s[i >> 2][i & 3] = 0;
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars.kv_full[s], 1);
@@ -197,6 +186,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const uint64_t dV = smem_desc(smem_u32(sm + kOffV), 16, 1024, kLayoutSW128);
     const uint64_t dL = smem_desc(smem_u32(sm + kOffL), 128, 256, kLayoutNone);
     const uint64_t dMu = smem_desc(smem_u32(sm + kOffMu), 128, 256, kLayoutNone);
+    unsigned long long nskip = 0;   // Skip Softmax: PVs skipped by this CTA
     bool ok = mbar_wait_warp(&bars.q_full, 0, &abort_s, p.st, lim, 200);
     ok = ok && mbar_wait_warp(&bars.kv_full[0], 0, &abort_s, p.st, lim, 201);
     if (ok) {
@@ -219,8 +209,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         if (!ok) break;
         tc_fence_after();
         const uint32_t sft = tmem + t * 128;   // scale vectors live in the consumed S_t columns
-        // (the flag was written before the warpgroup's p_full arrivals)
-        const bool skip_pv = SKIP && *reinterpret_cast<volatile int*>(&pv_skip_s[t]) != 0;
+        // (the flags were written before the warpgroup's p_full arrivals)
+        bool skip_pv = false;
+        if (SKIP) {
+          const volatile int* f = warp_drop_s[t];
+          skip_pv = f[0] && f[1] && f[2] && f[3];
+          nskip += skip_pv ? 1 : 0;
+        }
         if (!skip_pv) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)   // P_t at S_t columns 8..39, 8 columns (32 codes) per K step
@@ -254,6 +249,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       }
     }
     tc_commit_w(&bars.mma_done);
+    if (SKIP && lane == 0 && p.skipped && nskip) atomicAdd(p.skipped, nskip);
   } else if (warp == 2) {
     // ------------------------------------------------------------ block means -> fp32 [d][8] tiles
     const uint16_t* vm = p.v_mean + (int64_t)bh * nb * 128;
@@ -291,7 +287,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     int nref = 0;
     bool have_ref = false;
     float zrun = -INFINITY;        // Skip Softmax: running maximum of the block maxima (log2 units)
-    unsigned long long nskip = 0;
     float ltot = 0.0f;
     bool ok = true;
     // the next tile's K scale and V exponent are loaded one tile ahead, off the
@@ -306,9 +301,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         vex_next = __ldg(vex + j + 1);
       }
       ok = mbar_wait_warp(&bars.s_full[t], j & 1, &abort_s, p.st, lim, 400 + t);
-      // with SKIP the warpgroup votes below through named barriers, so its four
-      // warps must leave the loop together
-      if (SKIP) ok = wg_and(ok, 1 + t);
       if (!ok) break;
       tc_fence_after();
       float sv[128];
@@ -365,14 +357,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       // ExpCast: code = rne(s*c8 + 87 - 8*nref) via the magic-number FMA (two
       // scores per fma.rn.f32x2), clamped below at 0; the decoded probability is
       // float(code << 20) * 2^120, summed exactly enough in fp32 pairs
-      const bool tile_skip = SKIP && wg_and(rej, 1 + t);
+      const bool warp_drop = SKIP && __all_sync(0xffffffffu, rej);
       // a dropped row writes code 0 everywhere: multiplier 0, addend the bare magic constant
       const float badd = rej ? kMagic : kMagic + (float)(87 - 8 * nref);
       const float c8r = rej ? 0.0f : c8;
       const float2 c8x2 = make_float2(c8r, c8r), baddx2 = make_float2(badd, badd);
       float2 lsa = make_float2(0.0f, 0.0f), lsb = make_float2(0.0f, 0.0f);
       uint32_t pw[32];   // the row's 128 codes, 4 per word, in key order
-      if (!tile_skip) {
+      if (warp_drop) {
+        // PV may still run for the other warps' rows: these rows contribute zeros
+        const uint32_t zero[32] = {};
+        VCA_TMEM_ST32(tS + 8, zero);
+      } else {
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
         const int c = q * 4;
@@ -424,7 +420,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       }
       ltot = ltot * rescale + l;
       // UE8M0 scale vectors for this PV: A = 2^0, B = 2^v_exp[j]
-      if (!tile_skip) {
+      {
         const uint32_t eb = (uint32_t)(127 + vex_j);
         uint32_t sf[8];
 #pragma unroll
@@ -433,16 +429,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         for (int i = 4; i < 8; ++i) sf[i] = eb * 0x01010101u;
         tmem_st8(tS, sf);
       }
-      if (SKIP && r == 0) {
-        pv_skip_s[t] = tile_skip ? 1 : 0;
-        nskip += tile_skip ? 1 : 0;
-      }
+      if (SKIP && lane == 0) warp_drop_s[t][warp & 3] = warp_drop ? 1 : 0;
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&bars.p_full[t]);
     }
-    if (SKIP && r == 0 && p.skipped && nskip) atomicAdd(p.skipped, nskip);
     // ------------------------------------------------------------ epilogue
     if (ok) ok = mbar_wait_warp(&bars.o_done[t], (nkv - 1) & 1, &abort_s, p.st, lim, 420 + t);
     if (ok) {
