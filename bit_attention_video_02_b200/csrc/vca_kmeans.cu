@@ -23,7 +23,6 @@
 namespace vca {
 
 constexpr int kAssignThreads = 128;
-constexpr int kAccumChunk = 2048;   // tokens per accumulate CTA
 constexpr int kSortChunk = 1024;    // tokens per sort CTA
 
 struct KmWs {
@@ -32,6 +31,7 @@ struct KmWs {
   int* counts;       // [BH][k]
   int* ccount;       // [BH][nchunk][k]  per-chunk histogram
   int* cbase;        // [BH][nchunk][k]  scatter base per (chunk, cluster)
+  int* cstart;       // [BH][k]          first sorted position of each cluster
 };
 
 static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -51,6 +51,8 @@ static KmWs carve(void* ws, int BH, int N, int k, size_t* total) {
   off += align256((size_t)BH * nchunk * k * sizeof(int));
   w.cbase = (int*)(base + off);
   off += align256((size_t)BH * nchunk * k * sizeof(int));
+  w.cstart = (int*)(base + off);
+  off += align256((size_t)BH * k * sizeof(int));
   *total = off;
   return w;
 }
@@ -157,18 +159,18 @@ __global__ void __launch_bounds__(kAssignThreads) km_assign_kernel(const uint16_
   assign[(int64_t)bh * N + n] = best;
 }
 
-// Exact fixed-point sums per (cluster, channel) for one chunk of tokens.
-// Each warp takes one token at a time, lane l holding channels l + 32j.  The fixed-point value llrint(v * 2^24)
-// (|v| < 2^20, so it has at most 45 bits) is split exactly as hi * 2^22 + lo
-// with |hi|, |lo| < 2^22 using float operations only: f = v * 2^24 is exact,
-// hi = trunc(f / 2^22), lo = rne(f - hi * 2^22) (the only rounding, the same
-// as llrint's), each turned into an integer with the magic-number add.  The
-// halves go into 32-bit shared tables with shared-memory atomics; after every
-// 512 tokens (|sum| < 512 * 2^22 = 2^31, no overflow) they are folded into
-// int64 totals.  Integer addition is exact and order-free, so the result is
-// the exact sum whatever order the warps run in.
-constexpr int kAccumWarps = 8;
-constexpr int kAccumSub = 512;   // tokens between folds of the 32-bit halves
+// Exact fixed-point sums per (cluster, channel), walking the tokens in sorted
+// (cluster-contiguous) order.  Each warp takes kSegTok consecutive sorted
+// positions, lane l holding channels l + 32j.  llrint(v * 2^24) (|v| < 2^20, at
+// most 45 bits) is split exactly into hi * 2^22 + lo with |hi|, |lo| < 2^22 by
+// float operations only: f = v * 2^24 is exact, hi = trunc(f / 2^22),
+// lo = rne(f - hi * 2^22) (the only rounding, the same as llrint's), each made
+// an integer with the magic-number add.  The halves are summed in 32-bit
+// registers (at most kSegTok < 512 terms, so |sum| < 2^31) and flushed as one
+// int64 atomic per channel whenever the walk leaves a cluster.  Integer
+// addition is exact and order-free: the sums are exact whatever the order.
+constexpr int kSegTok = 256;   // sorted positions per warp
+constexpr int kSegWarps = 8;
 __device__ __forceinline__ void fix24_split(float v, int& hi, int& lo) {
   const float kMagic = 12582912.0f;   // 1.5 * 2^23
   const float f = v * 16777216.0f;
@@ -177,74 +179,74 @@ __device__ __forceinline__ void fix24_split(float v, int& hi, int& lo) {
   hi = (int)(__float_as_uint(hf + kMagic) - 0x4B400000u);
   lo = (int)(__float_as_uint(lf + kMagic) - 0x4B400000u);
 }
-__global__ void __launch_bounds__(kAccumWarps * 32) km_accum_kernel(const uint16_t* __restrict__ V,
-                                                                   const int32_t* __restrict__ assign,
-                                                                   long long* __restrict__ sums,
-                                                                   int* __restrict__ counts, int N, int k) {
-  extern __shared__ long long tot[];   // [k][128] int64, then hi[k][128], lo[k][128] int32
-  int* shi = reinterpret_cast<int*>(tot + k * 128);
-  int* slo = shi + k * 128;
-  __shared__ int cnt[VCA_MAX_CLUSTERS];
+__global__ void __launch_bounds__(kSegWarps * 32) km_accum_kernel(const uint16_t* __restrict__ V,
+                                                                 const int32_t* __restrict__ perm,
+                                                                 const int* __restrict__ cstart,
+                                                                 const int* __restrict__ counts,
+                                                                 long long* __restrict__ sums, int N, int k) {
+  __shared__ int cs[VCA_MAX_CLUSTERS], ce[VCA_MAX_CLUSTERS];
   const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < k * 128; i += blockDim.x) {
-    tot[i] = 0;
-    shi[i] = 0;
-    slo[i] = 0;
+  if (threadIdx.x < k) {
+    cs[threadIdx.x] = cstart[(int64_t)bh * k + threadIdx.x];
+    ce[threadIdx.x] = cs[threadIdx.x] + counts[(int64_t)bh * k + threadIdx.x];
   }
-  if (threadIdx.x < k) cnt[threadIdx.x] = 0;
   __syncthreads();
-  const int n0 = blockIdx.x * kAccumChunk, n1 = min(N, n0 + kAccumChunk);
+  const int q0 = (blockIdx.x * kSegWarps + warp) * kSegTok;
+  if (q0 >= N) return;
+  const int q1 = min(N, q0 + kSegTok);
+  // the cluster holding sorted position q0 (exactly one non-empty range contains it)
+  int found = -1;
+  for (int c2 = lane; c2 < k; c2 += 32)
+    if (cs[c2] <= q0 && q0 < ce[c2]) found = c2;
+  int c = max(__reduce_max_sync(0xffffffffu, found), 0);
+  int cend = ce[c];
   const uint16_t* vb = V + (int64_t)bh * N * 128;
-  const int32_t* ab = assign + (int64_t)bh * N;
-  for (int s0 = n0; s0 < n1; s0 += kAccumSub) {
-    const int s1 = min(n1, s0 + kAccumSub);
-    // two tokens per warp per step so that their loads overlap; lane l takes
-    // channels l, l+32, l+64, l+96 (64-byte coalesced loads, and the shared
-    // tables are hit one bank per lane)
-    for (int n = s0 + warp; n < s1; n += 2 * kAccumWarps) {
-      const int nbk = n + kAccumWarps;
-      const bool hb = nbk < s1;
-      const int a0 = __ldg(ab + n), a1 = hb ? __ldg(ab + nbk) : 0;
-      const uint16_t* r0 = vb + (int64_t)n * 128 + lane;
-      const uint16_t* r1 = vb + (int64_t)(hb ? nbk : n) * 128 + lane;
-      uint16_t x0[4], x1[4];
+  const int32_t* pb = perm + (int64_t)bh * N;
+  unsigned long long* sb = reinterpret_cast<unsigned long long*>(sums + (int64_t)bh * k * 128);
+  int hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
+  auto flush = [&]() {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        x0[j] = __ldg(r0 + 32 * j);
-        x1[j] = __ldg(r1 + 32 * j);
+    for (int j = 0; j < 4; ++j) {
+      const long long v = ((long long)hi[j] << 22) + (long long)lo[j];
+      if (v != 0) atomicAdd(sb + c * 128 + lane + 32 * j, (unsigned long long)v);
+      hi[j] = 0;
+      lo[j] = 0;
+    }
+  };
+  for (int base = q0; base < q1; base += 32) {
+    const int cnt = min(32, q1 - base);
+    const int myn = lane < cnt ? __ldg(pb + base + lane) : 0;
+    for (int i = 0; i < cnt; i += 4) {
+      // four tokens' rows in flight at once
+      uint16_t x[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int n = __shfl_sync(0xffffffffu, myn, (i + u) & 31);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) x[u][j] = i + u < cnt ? __ldg(vb + (int64_t)n * 128 + lane + 32 * j) : (uint16_t)0;
       }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int ch = lane + 32 * j;
-        int hi, lo;
-        fix24_split(__uint_as_float((uint32_t)x0[j] << 16), hi, lo);
-        if (hi) atomicAdd(shi + a0 * 128 + ch, hi);
-        atomicAdd(slo + a0 * 128 + ch, lo);
-        if (hb) {
-          fix24_split(__uint_as_float((uint32_t)x1[j] << 16), hi, lo);
-          if (hi) atomicAdd(shi + a1 * 128 + ch, hi);
-          atomicAdd(slo + a1 * 128 + ch, lo);
+      for (int u = 0; u < 4; ++u) {
+        if (i + u >= cnt) break;
+        const int q = base + i + u;
+        if (q >= cend) {   // the walk enters the next non-empty cluster
+          flush();
+          do {
+            ++c;
+          } while (c < k - 1 && ce[c] == cs[c]);
+          cend = ce[c];
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          int h, l;
+          fix24_split(__uint_as_float((uint32_t)x[u][j] << 16), h, l);
+          hi[j] += h;
+          lo[j] += l;
         }
       }
-      if (lane == 0) {
-        atomicAdd(&cnt[a0], 1);
-        if (hb) atomicAdd(&cnt[a1], 1);
-      }
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < k * 128; i += blockDim.x) {
-      tot[i] += ((long long)shi[i] << 22) + (long long)slo[i];
-      shi[i] = 0;
-      slo[i] = 0;
-    }
-    __syncthreads();
   }
-  long long* dst = sums + (int64_t)bh * k * 128;
-  for (int i = threadIdx.x; i < k * 128; i += blockDim.x) {
-    const long long s = tot[i];
-    if (s != 0) atomicAdd(reinterpret_cast<unsigned long long*>(dst + i), (unsigned long long)s);
-  }
-  if (threadIdx.x < k && cnt[threadIdx.x] != 0) atomicAdd(counts + (int64_t)bh * k + threadIdx.x, cnt[threadIdx.x]);
+  flush();
 }
 
 __global__ void km_update_kernel(const long long* __restrict__ sums, const int* __restrict__ counts,
@@ -272,8 +274,8 @@ __global__ void sort_count_kernel(const int32_t* __restrict__ assign, int* __res
 
 // One CTA per head: base(chunk, c) = sum of all tokens of clusters < c plus the
 // tokens of cluster c in earlier chunks.
-__global__ void sort_scan_kernel(const int* __restrict__ ccount, int* __restrict__ cbase, int k,
-                                 int nchunk) {
+__global__ void sort_scan_kernel(const int* __restrict__ ccount, int* __restrict__ cbase,
+                                 int* __restrict__ counts, int* __restrict__ cstart, int k, int nchunk) {
   __shared__ int tot[VCA_MAX_CLUSTERS];
   __shared__ int off[VCA_MAX_CLUSTERS];
   const int bh = blockIdx.x, c = threadIdx.x;
@@ -294,6 +296,8 @@ __global__ void sort_scan_kernel(const int* __restrict__ ccount, int* __restrict
   }
   __syncthreads();
   if (c < k) {
+    counts[(int64_t)bh * k + c] = tot[c];
+    cstart[(int64_t)bh * k + c] = off[c];
     int run = off[c];
     for (int j = 0; j < nchunk; ++j) {
       cb[j * k + c] = run;
@@ -349,40 +353,39 @@ static int cluster_permute_impl(const vca_bf16* V, int B, int H, int N, int d, i
                                 const KmWs& w, cudaStream_t s) {
   const int BH = B * H;
   size_t sums_bytes = (size_t)BH * k * 128 * sizeof(long long);
-  size_t counts_bytes = (size_t)BH * k * sizeof(int);
   km_init_kernel<<<dim3(BH, k), 128, 0, s>>>(V, init, cent, N, k);
   int rc = check_launch("km_init_kernel");
   if (rc) return rc;
   // centroid table padded to 16 or 32 pairs (pads sit at infinity)
   const int np = (k + 1) / 2 <= 16 ? 16 : 32;
   const size_t assign_smem = (size_t)np * 128 * sizeof(float2);
-  const size_t accum_smem = (size_t)k * 128 * (sizeof(long long) + 2 * sizeof(int));
   auto assign_kernel = np == 16 ? km_assign_kernel<16> : km_assign_kernel<32>;
   if (cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)assign_smem) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(km_accum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)accum_smem) !=
-          cudaSuccess)
+      cudaSuccess)
     return fail(VCA_ERR_CUDA, "vca_cluster_permute: cannot set shared-memory size");
   const dim3 g_assign((N + 2 * kAssignThreads - 1) / (2 * kAssignThreads), BH);
-  const dim3 g_accum((N + kAccumChunk - 1) / kAccumChunk, BH);
+  const dim3 g_accum((N + kSegWarps * kSegTok - 1) / (kSegWarps * kSegTok), BH);
+  const int nchunk = (N + kSortChunk - 1) / kSortChunk;
+  // Every round: assign, stable counting sort by cluster (its scan also gives
+  // the cluster sizes and starts), exact sums along the sorted order, update.
+  // The last round's sort is the permutation the caller gets.
   for (int it = 0; it < iters; ++it) {
     assign_kernel<<<g_assign, kAssignThreads, assign_smem, s>>>(V, cent, assign, N, k);
     if ((rc = check_launch("km_assign_kernel"))) return rc;
-    if (cudaMemsetAsync(w.sums, 0, sums_bytes, s) != cudaSuccess ||
-        cudaMemsetAsync(w.counts, 0, counts_bytes, s) != cudaSuccess)
+    sort_count_kernel<<<dim3(nchunk, BH), 256, 0, s>>>(assign, w.ccount, N, k, nchunk);
+    if ((rc = check_launch("sort_count_kernel"))) return rc;
+    sort_scan_kernel<<<BH, 64, 0, s>>>(w.ccount, w.cbase, w.counts, w.cstart, k, nchunk);
+    if ((rc = check_launch("sort_scan_kernel"))) return rc;
+    sort_scatter_kernel<<<dim3(nchunk, BH), 32, 0, s>>>(assign, w.cbase, perm, N, k, nchunk);
+    if ((rc = check_launch("sort_scatter_kernel"))) return rc;
+    if (cudaMemsetAsync(w.sums, 0, sums_bytes, s) != cudaSuccess)
       return fail(VCA_ERR_CUDA, "vca_cluster_permute: memset failed");
-    km_accum_kernel<<<g_accum, kAccumWarps * 32, accum_smem, s>>>(V, assign, w.sums, w.counts, N, k);
+    km_accum_kernel<<<g_accum, kSegWarps * 32, 0, s>>>(V, perm, w.cstart, w.counts, w.sums, N, k);
     if ((rc = check_launch("km_accum_kernel"))) return rc;
     km_update_kernel<<<dim3(BH, k), 128, 0, s>>>(w.sums, w.counts, cent, k);
     if ((rc = check_launch("km_update_kernel"))) return rc;
   }
-  const int nchunk = (N + kSortChunk - 1) / kSortChunk;
-  sort_count_kernel<<<dim3(nchunk, BH), 256, 0, s>>>(assign, w.ccount, N, k, nchunk);
-  if ((rc = check_launch("sort_count_kernel"))) return rc;
-  sort_scan_kernel<<<BH, 64, 0, s>>>(w.ccount, w.cbase, k, nchunk);
-  if ((rc = check_launch("sort_scan_kernel"))) return rc;
-  sort_scatter_kernel<<<dim3(nchunk, BH), 32, 0, s>>>(assign, w.cbase, perm, N, k, nchunk);
-  return check_launch("sort_scatter_kernel");
+  return 0;
 }
 
 static int check_cluster_args(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
