@@ -1,0 +1,190 @@
+// vca_pipeline.cu -- the whole path from host buffers to host buffers, with the
+// host<->device copies overlapped with the kernels.
+//
+// A layer's (batch, head) units are independent ("VC-Attention: Training-Free
+// Low-Bit Attention Speeds Video Diffusion Up to 3.6x": grouping, quantisation
+// and attention are all per head), so the layer is cut into chunks of heads and
+// run as a three-stage pipeline over two device slots: copy chunk c+1 in while
+// chunk c is grouped, quantised and attended, and copy chunk c-1's output out.
+// Each chunk runs exactly the per-head kernels of vca_cluster_permute,
+// vca_smooth_quantize_qkv and vca_attention_fwd, so the result is the same, bit
+// for bit, as running the three calls on the whole layer.
+#include <mutex>
+
+#include "vca_host.h"
+
+using namespace vca;
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Byte layout of one device slot for a chunk of `u` (batch, head) units.
+struct Slot {
+  size_t q, k, v, o, cent, assign, perm, qq, kq, vrt, qs, ks, ve, vm, ws, total;
+};
+
+Slot slot_layout(int u, int N, int d, int k) {
+  const int nb = (N + 127) / 128;
+  const size_t Np = (size_t)nb * 128, un = (size_t)u * N;
+  Slot s;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  s.q = take(un * d * 2);
+  s.k = take(un * d * 2);
+  s.v = take(un * d * 2);
+  s.o = take(un * d * 2);
+  s.cent = take((size_t)u * k * d * 4);
+  s.assign = take(un * 4);
+  s.perm = take(un * 4);
+  s.qq = take((size_t)u * Np * d);
+  s.kq = take((size_t)u * Np * d);
+  s.vrt = take((size_t)u * Np * d);
+  s.qs = take((size_t)u * nb * 4);
+  s.ks = take((size_t)u * nb * 4);
+  s.ve = take((size_t)u * nb);
+  s.vm = take((size_t)u * nb * d * 2);
+  size_t ws = vca_cluster_permute_workspace_size(1, u, N, k);
+  ws = ws > vca_smooth_quantize_workspace_size(1, u, N) ? ws : vca_smooth_quantize_workspace_size(1, u, N);
+  ws = ws > vca_attention_workspace_size(1, u, N) ? ws : vca_attention_workspace_size(1, u, N);
+  s.ws = take(ws);
+  s.total = off;
+  return s;
+}
+
+// Three non-blocking streams per device, created on first use and kept for the
+// life of the process.
+struct Streams {
+  cudaStream_t h2d = nullptr, comp = nullptr, d2h = nullptr;
+};
+std::mutex g_streams_mu;
+Streams g_streams[64];
+
+int get_streams(Streams* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return fail(VCA_ERR_CUDA, "vca_vc_attention_host: no current device");
+  std::lock_guard<std::mutex> lock(g_streams_mu);
+  Streams& s = g_streams[dev];
+  if (!s.h2d) {
+    if (cudaStreamCreateWithFlags(&s.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&s.comp, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&s.d2h, cudaStreamNonBlocking) != cudaSuccess)
+      return fail(VCA_ERR_CUDA, "vca_vc_attention_host: cannot create streams");
+  }
+  *out = s;
+  return VCA_OK;
+}
+
+int units_per_chunk(int units, int heads_per_chunk) {
+  if (heads_per_chunk > 0) return heads_per_chunk < units ? heads_per_chunk : units;
+  const int u = (units + 7) / 8;   // about eight chunks
+  return u < 1 ? 1 : u;
+}
+
+}  // namespace
+
+extern "C" size_t vca_vc_attention_host_buffer_size(int B, int H, int N, int d, int k, int heads_per_chunk) {
+  if (B < 1 || H < 1 || N < 1 || d != VCA_HEAD_DIM || k < 1 || k > VCA_MAX_CLUSTERS) return 0;
+  const int u = units_per_chunk(B * H, heads_per_chunk);
+  return 2 * slot_layout(u, N, d, k).total;
+}
+
+extern "C" int vca_vc_attention_host(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V, int B, int H, int N,
+                                     int d, int k, int iters, float softmax_scale, vca_bf16* O, int heads_per_chunk,
+                                     void* dev_buf, size_t dev_bytes, vca_stream_t stream) {
+  const char* fn = "vca_vc_attention_host";
+  if (!Q || !K || !V || !O || !dev_buf) return fail(VCA_ERR_INVALID, "%s: null pointer", fn);
+  if (d != VCA_HEAD_DIM) return fail(VCA_ERR_UNSUPPORTED, "%s: d must be 128", fn);
+  if (B < 1 || H < 1 || N < 1 || k < 1 || k > VCA_MAX_CLUSTERS || iters < 1)
+    return fail(VCA_ERR_INVALID, "%s: bad shape or k-means arguments", fn);
+  if (heads_per_chunk < 0) return fail(VCA_ERR_INVALID, "%s: heads_per_chunk must be >= 0", fn);
+  const int units = B * H;
+  const int u = units_per_chunk(units, heads_per_chunk);
+  const Slot L = slot_layout(u, N, d, k);
+  if (dev_bytes < 2 * L.total) return fail(VCA_ERR_WORKSPACE, "%s: device buffer too small", fn);
+  Streams st;
+  int rc = get_streams(&st);
+  if (rc) return rc;
+
+  // the pipeline starts after the work already queued on the caller's stream
+  cudaEvent_t start, ev_in[2], ev_done[2], ev_free[2];
+  if (cudaEventCreateWithFlags(&start, cudaEventDisableTiming) != cudaSuccess)
+    return fail(VCA_ERR_CUDA, "%s: cannot create events", fn);
+  for (int i = 0; i < 2; ++i)
+    if (cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ev_done[i], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ev_free[i], cudaEventDisableTiming) != cudaSuccess)
+      return fail(VCA_ERR_CUDA, "%s: cannot create events", fn);
+  cudaEventRecord(start, (cudaStream_t)stream);
+  cudaStreamWaitEvent(st.h2d, start, 0);
+  cudaStreamWaitEvent(st.comp, start, 0);
+  cudaStreamWaitEvent(st.d2h, start, 0);
+
+  const size_t row = (size_t)N * d;   // elements per unit
+  char* base = (char*)dev_buf;
+  const int nchunks = (units + u - 1) / u;
+  // each call starts with clean status words in both slots' workspaces
+  for (int s = 0; s < 2 && !rc; ++s) rc = vca_reset_status(base + (size_t)s * L.total + L.ws, st.comp);
+  for (int c = 0; c < nchunks && !rc; ++c) {
+    const int s = c & 1;
+    const int u0 = c * u, uc = (u0 + u <= units) ? u : units - u0;
+    char* b = base + (size_t)s * L.total;
+    const size_t bytes = (size_t)uc * row * 2;
+    // slot s is free once chunk c-2's output has left the device
+    if (c >= 2) cudaStreamWaitEvent(st.h2d, ev_free[s], 0);
+    if (cudaMemcpyAsync(b + L.q, Q + (size_t)u0 * row, bytes, cudaMemcpyHostToDevice, st.h2d) != cudaSuccess ||
+        cudaMemcpyAsync(b + L.k, K + (size_t)u0 * row, bytes, cudaMemcpyHostToDevice, st.h2d) != cudaSuccess ||
+        cudaMemcpyAsync(b + L.v, V + (size_t)u0 * row, bytes, cudaMemcpyHostToDevice, st.h2d) != cudaSuccess) {
+      rc = fail(VCA_ERR_CUDA, "%s: host-to-device copy failed", fn);
+      break;
+    }
+    cudaEventRecord(ev_in[s], st.h2d);
+    cudaStreamWaitEvent(st.comp, ev_in[s], 0);
+    void* ws = b + L.ws;
+    const size_t wsb = L.total - L.ws;
+    vca_bf16* Vd = (vca_bf16*)(b + L.v);
+    rc = vca_cluster_permute(Vd, 1, uc, N, d, k, iters, nullptr, (float*)(b + L.cent), (int32_t*)(b + L.assign),
+                             (int32_t*)(b + L.perm), ws, wsb, st.comp);
+    if (!rc)
+      rc = vca_smooth_quantize_qkv((vca_bf16*)(b + L.q), (vca_bf16*)(b + L.k), Vd, (int32_t*)(b + L.perm), 1, uc,
+                                   N, d, 128, (uint8_t*)(b + L.qq), (float*)(b + L.qs), (uint8_t*)(b + L.kq),
+                                   (float*)(b + L.ks), (uint8_t*)(b + L.vrt), (int8_t*)(b + L.ve),
+                                   (vca_bf16*)(b + L.vm), ws, wsb, st.comp);
+    if (!rc)
+      rc = vca_attention_fwd((uint8_t*)(b + L.qq), (float*)(b + L.qs), (uint8_t*)(b + L.kq), (float*)(b + L.ks),
+                             (uint8_t*)(b + L.vrt), (int8_t*)(b + L.ve), (vca_bf16*)(b + L.vm), 1, uc, N, d,
+                             softmax_scale, (vca_bf16*)(b + L.o), nullptr, ws, wsb, st.comp);
+    if (rc) break;
+    cudaEventRecord(ev_done[s], st.comp);
+    cudaStreamWaitEvent(st.d2h, ev_done[s], 0);
+    if (cudaMemcpyAsync(O + (size_t)u0 * row, b + L.o, bytes, cudaMemcpyDeviceToHost, st.d2h) != cudaSuccess) {
+      rc = fail(VCA_ERR_CUDA, "%s: device-to-host copy failed", fn);
+      break;
+    }
+    cudaEventRecord(ev_free[s], st.d2h);
+  }
+  // blocking call: everything queued above has finished when it returns
+  const bool sync_ok = cudaStreamSynchronize(st.h2d) == cudaSuccess &&
+                       cudaStreamSynchronize(st.comp) == cudaSuccess &&
+                       cudaStreamSynchronize(st.d2h) == cudaSuccess;
+  cudaEventDestroy(start);
+  for (int i = 0; i < 2; ++i) {
+    cudaEventDestroy(ev_in[i]);
+    cudaEventDestroy(ev_done[i]);
+    cudaEventDestroy(ev_free[i]);
+  }
+  if (rc) return rc;
+  if (!sync_ok) return fail(VCA_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(cudaGetLastError()));
+  // device-side errors of either slot (timeouts, non-finite inputs)
+  for (int s = 0; s < 2 && s < nchunks; ++s) {
+    int where = 0, info = 0;
+    rc = vca_check_status(base + (size_t)s * L.total + L.ws, nullptr, &where, &info);
+    if (rc) return rc;
+  }
+  return VCA_OK;
+}

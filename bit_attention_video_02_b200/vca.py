@@ -33,7 +33,7 @@ EXPORTED = [
     "vca_smooth_quantize_workspace_size", "vca_smooth_quantize_qkv",
     "vca_attention_workspace_size", "vca_attention_fwd",
     "vca_bf16_attention_workspace_size", "vca_bf16_attention_fwd", "vca_schedule_regroup",
-    "vca_attention_fwd_skip",
+    "vca_attention_fwd_skip", "vca_vc_attention_host_buffer_size", "vca_vc_attention_host",
 ]
 
 
@@ -73,11 +73,14 @@ def lib() -> ctypes.CDLL:
         L.vca_bf16_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
         L.vca_schedule_regroup.argtypes = [i32, i32, i32, f32]
         L.vca_attention_fwd_skip.argtypes = [vp] * 7 + [i32, i32, i32, i32, f32, f32, vp, vp, vp, vp, sz, vp]
+        L.vca_vc_attention_host_buffer_size.restype = sz
+        L.vca_vc_attention_host_buffer_size.argtypes = [i32] * 6
+        L.vca_vc_attention_host.argtypes = [vp, vp, vp] + [i32] * 6 + [f32, vp, i32, vp, sz, vp]
         for fn in ("vca_reset_status", "vca_check_status", "vca_debug_wait_timeout", "vca_expcast_ref",
                    "vca_e4m3_encode", "vca_cluster_permute", "vca_cluster_permute_noalloc",
                    "vca_smooth_quantize_qkv",
                    "vca_attention_fwd", "vca_bf16_attention_fwd", "vca_schedule_regroup",
-                   "vca_attention_fwd_skip"):
+                   "vca_attention_fwd_skip", "vca_vc_attention_host"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -305,3 +308,34 @@ class VCAttentionLayer:
             self.regrouped_at.append(step)
         ops = smooth_quantize(Q, K, V, self.perm, ws=self.ws, stream=stream)
         return attention_fwd(ops, Q.shape[2], softmax_scale, ws=self.ws, stream=stream)
+
+
+_host_bufs = {}
+
+
+def vc_attention_host(Q, K, V, k: int = 32, iters: int = 3, softmax_scale=None, O=None, heads_per_chunk: int = 0,
+                      device=None, stream=None):
+    """vca_vc_attention_host: the whole path from host (CPU) bf16 tensors to a
+    host bf16 output, copies overlapped with the kernels.  Pass page-locked
+    tensors (tensor.pin_memory()) for the overlap.  The device scratch is kept
+    per (device, size) between calls."""
+    assert Q.device.type == "cpu" and Q.dtype == torch.bfloat16 and Q.is_contiguous()
+    assert K.shape == Q.shape == V.shape and K.is_contiguous() and V.is_contiguous()
+    B, H, N, d = Q.shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    if O is None:
+        O = torch.empty(Q.shape, dtype=torch.bfloat16, pin_memory=Q.is_pinned())
+    need = lib().vca_vc_attention_host_buffer_size(B, H, N, d, k, heads_per_chunk)
+    if need == 0:
+        raise VcaError(ERR_INVALID, "vc_attention_host: unsupported shape")
+    key = (dev.index, need)
+    if key not in _host_bufs:
+        _host_bufs.clear()
+        _host_bufs[key] = torch.empty(need, dtype=torch.uint8, device=dev)
+    buf = _host_bufs[key]
+    with torch.cuda.device(dev):
+        _check(lib().vca_vc_attention_host(_ptr(Q), _ptr(K), _ptr(V), B, H, N, d, k, iters, scale, _ptr(O),
+                                           heads_per_chunk, ctypes.c_void_p(buf.data_ptr()), need,
+                                           _stream(stream)))
+    return O

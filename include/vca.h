@@ -232,6 +232,30 @@ int vca_attention_fwd_skip(const uint8_t* Qq, const float* q_scale, const uint8_
                            unsigned long long* skipped_tiles, void* ws, size_t ws_bytes,
                            vca_stream_t stream);
 
+/* The whole path from host buffers to host buffers (grouping with
+ * vca_cluster_permute from its default initialisation, vca_smooth_quantize_qkv,
+ * vca_attention_fwd), with the copies overlapped with the kernels.  The pages
+ * have no counterpart: it serves callers whose activations live in host memory.
+ * (b, h) units are independent, so the layer runs in chunks of
+ * `heads_per_chunk` units (0 = about eight chunks) through a three-stage
+ * pipeline on library-owned streams over two device slots: copy chunk c+1 in,
+ * compute chunk c, copy chunk c-1 out.  Results equal the three calls on the
+ * whole layer bit for bit.
+ *   Q, K, V   [B][H][N][d] bf16, HOST memory (in); page-locked memory
+ *             (cudaHostAlloc / cudaHostRegister) is needed for the copies to
+ *             overlap -- pageable memory works but serialises them
+ *   O         [B][H][N][d] bf16, HOST memory (out)
+ *   dev_buf   device scratch of vca_vc_attention_host_buffer_size() bytes,
+ *             owned by the caller; its contents need no initialisation
+ *   stream    the pipeline starts after the work queued on `stream`
+ * Blocking: returns once O is written, with the first error of the host
+ * checks, the launches or the device status words (bounded waits, non-finite
+ * input).  d must be 128; 1 <= k <= VCA_MAX_CLUSTERS; iters >= 1. */
+size_t vca_vc_attention_host_buffer_size(int B, int H, int N, int d, int k, int heads_per_chunk);
+int vca_vc_attention_host(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V, int B, int H, int N,
+                          int d, int k, int iters, float softmax_scale, vca_bf16* O, int heads_per_chunk,
+                          void* dev_buf, size_t dev_bytes, vca_stream_t stream);
+
 /* In-repo BF16 comparator: exact-softmax flash attention (online softmax with
  * exp2), tcgen05 BF16 MMAs with fp32 accumulation in tensor memory.
  *   Q, K, V, O [B][H][N][d] bf16; lse [B][H][N] fp32 natural log (nullable). */
