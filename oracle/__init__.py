@@ -71,6 +71,8 @@ def _declare(L):
     L.vo_smooth_quantize_head.argtypes = [vp] * 4 + [i32, i32] + [vp] * 7
     L.vo_attention_head.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, vp, vp, vp]
     L.vo_attention_head_bf16.argtypes = [vp] * 4 + [i32, i32, f64, vp, i32, i32, vp]
+    L.vo_sage_quantize_head.argtypes = [vp] * 3 + [i32, i32] + [vp] * 7
+    L.vo_attention_head_sage.argtypes = [vp] * 6 + [i32, i32, f64, vp, i32, i32, vp, vp]
     L.vo_attention_head_skip.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, f64, vp, vp, vp]
     L.vo_attention_head_bf16_skip.argtypes = [vp] * 4 + [i32, i32, f64, vp, i32, i32, f64, vp]
     L.vo_exact_attention_head.argtypes = [vp] * 3 + [i32, i32, f64, vp, i32, vp]
@@ -175,6 +177,23 @@ def smooth_quantize_head(Q, K, V, perm):
     return out
 
 
+def sage_quantize_head(Q, K, V):
+    """One head of the SAGE-style comparison quantisation (per-token Q,
+    per-16-token K after K-mean smoothing, per-channel V; no reordering)."""
+    Q, K, V = (np.ascontiguousarray(a, dtype=np.uint16) for a in (Q, K, V))
+    N, d = Q.shape
+    Np = (N + BLOCK - 1) // BLOCK * BLOCK
+    out = dict(
+        Qq=np.zeros((Np, d), np.uint8), q_scale=np.empty(Np, np.float32),
+        Kq=np.zeros((Np, d), np.uint8), k_scale=np.empty(Np // 16, np.float32),
+        VcT=np.zeros((d, Np), np.uint8), v_chscale=np.empty(d, np.float32),
+        k_mean=np.empty(d, np.uint16))
+    lib().vo_sage_quantize_head(
+        _p(Q), _p(K), _p(V), N, d, _p(out["Qq"]), _p(out["q_scale"]), _p(out["Kq"]), _p(out["k_scale"]),
+        _p(out["VcT"]), _p(out["v_chscale"]), _p(out["k_mean"]))
+    return out
+
+
 # ------------------------------------------------------------------ attention
 def _rows(rows, N):
     if rows is None:
@@ -210,6 +229,20 @@ def attention_head_bf16(Q, K, V, perm, softmax_scale: float, rows=None, flags: i
     lib().vo_attention_head_bf16_skip(_p(Q), _p(K), _p(V), _p(perm), N, d, float(softmax_scale),
                                       _p(rows), rows.shape[0], int(flags), float(skip_lambda), _p(O))
     return O
+
+
+def attention_head_sage(ops: dict, N: int, softmax_scale: float, rows=None, flags: int = 0):
+    """Attention on SAGE-style operands (dict from ``sage_quantize_head``).
+    Returns (O [nrows, d] fp64, lse [nrows])."""
+    rows = _rows(rows, N)
+    d = ops["Qq"].shape[1]
+    O = np.empty((rows.shape[0], d), np.float64)
+    lse = np.empty(rows.shape[0], np.float64)
+    c = {k: np.ascontiguousarray(v) for k, v in ops.items()}
+    lib().vo_attention_head_sage(
+        _p(c["Qq"]), _p(c["q_scale"]), _p(c["Kq"]), _p(c["k_scale"]), _p(c["VcT"]), _p(c["v_chscale"]),
+        N, d, float(softmax_scale), _p(rows), rows.shape[0], int(flags), _p(O), _p(lse))
+    return O, lse
 
 
 def exact_attention_head(Q, K, V, softmax_scale: float, rows=None):

@@ -322,6 +322,73 @@ void vo_smooth_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_
     }
 }
 
+/* SAGE-style quantisation, the comparison recipe of "Accelerating Video
+ * Generation with GEMM Quantization, Attention Quantization and Skip Softmax
+ * Attention in TensorRT-LLM" (section "Quantized Attention": q_block_size 1,
+ * k_block_size 16, v_block_size 1, FP8 V), with K smoothed by its channel
+ * mean (SageAttention2's K smoothing, named there as the line of work
+ * followed).  No reordering, no block means:
+ *   k_mean[c]  = bf16(exact mean of K[:, c] over all N tokens) (fixed-point
+ *                sum, one fp64 division, one rounding -- as the V block mean)
+ *   K' = K - k_mean (fp32); Q and K' get one fp32 scale per group (1 token
+ *   for Q, 16 tokens for K'): amax / 448, codes e4m3(x * (448 / amax));
+ *   V gets one fp32 scale per channel over all N tokens, same formula;
+ *   VcT[c][j] = code of V[j][c] (channel-major, padded to Np with 0).
+ *   q_scale [Np], k_scale [Np/16], v_chscale [d]; an all-zero group has
+ *   scale 1 and codes 0. */
+static void quant_group(const float* x, int n, uint8_t* out, float* scale) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i)
+        if (fabsf(x[i]) > amax) amax = fabsf(x[i]);
+    if (!(amax > 0.0f)) {
+        *scale = 1.0f;
+        memset(out, 0, (size_t)n);
+        return;
+    }
+    *scale = amax / 448.0f;
+    float inv = 448.0f / amax;
+    for (int i = 0; i < n; ++i) out[i] = vo_e4m3_encode(x[i] * inv);
+}
+
+void vo_sage_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int N, int d,
+                           uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                           uint8_t* VcT, float* v_chscale, uint16_t* k_mean) {
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    int64_t Np = (int64_t)nb * VO_BLOCK;
+    memset(Qq, 0, (size_t)Np * d);
+    memset(Kq, 0, (size_t)Np * d);
+    memset(VcT, 0, (size_t)Np * d);
+    for (int64_t j = 0; j < Np; ++j) q_scale[j] = 1.0f;
+    for (int64_t g = 0; g < Np / 16; ++g) k_scale[g] = 1.0f;
+    float* x = (float*)malloc((size_t)16 * d * sizeof(float));
+    for (int c = 0; c < d; ++c) {
+        int64_t S = 0;
+        for (int j = 0; j < N; ++j) S += llrint((double)vo_bf16_to_float(K[(int64_t)j * d + c]) * 16777216.0);
+        k_mean[c] = vo_double_to_bf16_rne((double)S / ((double)N * 16777216.0));
+    }
+    for (int j = 0; j < N; ++j) {
+        for (int c = 0; c < d; ++c) x[c] = vo_bf16_to_float(Q[(int64_t)j * d + c]);
+        quant_group(x, d, Qq + (int64_t)j * d, &q_scale[j]);
+    }
+    for (int g = 0; g * 16 < N; ++g) {
+        int n = N - g * 16 < 16 ? N - g * 16 : 16;
+        for (int t = 0; t < n; ++t)
+            for (int c = 0; c < d; ++c)
+                x[t * d + c] = vo_bf16_to_float(K[(int64_t)(g * 16 + t) * d + c]) - vo_bf16_to_float(k_mean[c]);
+        quant_group(x, n * d, Kq + (int64_t)g * 16 * d, &k_scale[g]);
+    }
+    float* col = (float*)malloc((size_t)N * sizeof(float));
+    uint8_t* cc = (uint8_t*)malloc((size_t)N);
+    for (int c = 0; c < d; ++c) {
+        for (int j = 0; j < N; ++j) col[j] = vo_bf16_to_float(V[(int64_t)j * d + c]);
+        quant_group(col, N, cc, &v_chscale[c]);
+        memcpy(VcT + (int64_t)c * Np, cc, (size_t)N);
+    }
+    free(x);
+    free(col);
+    free(cc);
+}
+
 /* --------------------------------------------------------------- attention */
 
 /* The ExpCast max grid: m = phi + n with integer n and phi = 0.65/8, so that
@@ -490,6 +557,37 @@ void vo_attention_head_skip(const uint8_t* Qq, const float* q_scale, const uint8
     }
     attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, skip_log2_of(skip_lambda), O,
               lse, lblk);
+    free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
+}
+
+/* Attention on SAGE-style operands: the same row algorithm (ExpCast codes,
+ * online reference) with per-token Q scales, per-16-key K scales, no V block
+ * exponents or means, and output channel c multiplied by v_chscale[c]. */
+void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                            const float* k_scale, const uint8_t* VcT, const float* v_chscale,
+                            int N, int d, double softmax_scale, const int32_t* rows, int nrows,
+                            int flags, double* O, double* lse) {
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    int64_t Np = (int64_t)nb * VO_BLOCK;
+    double* qh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* kh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* rh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* qs = (double*)malloc((size_t)N * sizeof(double));
+    double* ks = (double*)malloc((size_t)N * sizeof(double));
+    double* mu = (double*)calloc((size_t)nb * d, sizeof(double));
+    int* ve = (int*)calloc((size_t)nb, sizeof(int));
+    for (int j = 0; j < N; ++j) {
+        qs[j] = q_scale[j];
+        ks[j] = k_scale[j / 16];
+        for (int c = 0; c < d; ++c) {
+            qh[(int64_t)j * d + c] = vo_e4m3_decode(Qq[(int64_t)j * d + c]);
+            kh[(int64_t)j * d + c] = vo_e4m3_decode(Kq[(int64_t)j * d + c]);
+            rh[(int64_t)j * d + c] = vo_e4m3_decode(VcT[(int64_t)c * Np + j]);
+        }
+    }
+    attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, -INFINITY, O, lse, NULL);
+    for (int r = 0; r < nrows; ++r)
+        for (int c = 0; c < d; ++c) O[(int64_t)r * d + c] *= v_chscale[c];
     free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
 }
 

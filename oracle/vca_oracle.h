@@ -96,6 +96,18 @@ void vo_attention_head_skip(const uint8_t* Qq, const float* q_scale, const uint8
                             const int32_t* rows, int nrows, int flags, double skip_lambda,
                             double* O, double* lse, double* lblk);
 
+/* SAGE-style comparison recipe (TensorRT-LLM video post, section "Quantized
+ * Attention": per-token Q scales, one K scale per 16 tokens after K-mean
+ * smoothing, per-channel FP8 V; no reordering, no block means).
+ * q_scale [Np], k_scale [Np/16], VcT [d][Np], v_chscale [d], k_mean [d] bf16. */
+void vo_sage_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int N, int d,
+                           uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                           uint8_t* VcT, float* v_chscale, uint16_t* k_mean);
+void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                            const float* k_scale, const uint8_t* VcT, const float* v_chscale,
+                            int N, int d, double softmax_scale, const int32_t* rows, int nrows,
+                            int flags, double* O, double* lse);
+
 /* Same algorithm, straight from bf16 Q/K/V and a permutation; with
  * VO_IDENTITY_QUANT the quantisers are the identity (for reductions). */
 void vo_attention_head_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t* V,

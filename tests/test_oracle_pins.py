@@ -523,3 +523,75 @@ def test_skip_softmax_zero_lambda_is_the_plain_algorithm():
                                        skip_lambda=2.0 ** -6)
     keep = _survivors(Q, K, 1 / math.sqrt(128), 2.0 ** -6, rows)[:, ::128]
     assert np.all(lblk[~keep] == 0.0) and np.all(lblk[keep] > 0.0)
+
+
+# ------------------------------------------------------------------ SAGE-style comparison recipe
+def _e4m3_table():
+    return np.array([oracle.lib().vo_e4m3_decode(i) for i in range(256)], np.float64)
+
+
+def _e4m3_err_bound(x_scaled):
+    # round-to-nearest E4M3: half an ulp, i.e. 2^(e-4) for normal values and
+    # 2^-10 in the subnormal range (scaled units); the 1e-4 slack covers the
+    # fp32 scale product (x * (448/amax) is rounded in fp32 before encoding,
+    # so a value the fp64 check places just past a midpoint may sit on it)
+    e = np.floor(np.log2(np.maximum(np.abs(x_scaled), 2.0 ** -6)))
+    return np.ldexp(1.0, (e - 4).astype(int)) * (1.0 + 1e-4)
+
+
+def test_sage_quantisers_follow_their_definition():
+    rng = np.random.default_rng(41)
+    N = 300
+    Q, K, V = _bits(rng, N), _bits(rng, N), _bits(rng, N)
+    ops = oracle.sage_quantize_head(Q, K, V)
+    dec = _e4m3_table()
+    qf, kf, vf = (bits_to_f32(a).astype(np.float64) for a in (Q, K, V))
+    # K mean: exact mean over all tokens, rounded once to bf16
+    want_mean = bf16_bits_of(kf.mean(0).astype(np.float64))
+    assert np.array_equal(ops["k_mean"], want_mean)
+    km = bits_to_f32(ops["k_mean"]).astype(np.float64)
+    # Q: one scale per token
+    assert np.allclose(ops["q_scale"][:N], np.abs(qf).max(1).astype(np.float32) / np.float32(448), rtol=0, atol=0)
+    qrec = dec[ops["Qq"][:N]] * ops["q_scale"][:N, None]
+    assert np.all(np.abs(qrec - qf) <= _e4m3_err_bound(qf / ops["q_scale"][:N, None]) * ops["q_scale"][:N, None])
+    # K: smoothed, one scale per 16 tokens
+    ks = np.repeat(ops["k_scale"], 16)[:N, None].astype(np.float64)
+    kp = (kf.astype(np.float32) - km.astype(np.float32)).astype(np.float64)
+    krec = dec[ops["Kq"][:N]] * ks
+    assert np.all(np.abs(krec - kp) <= _e4m3_err_bound(kp / ks) * ks)
+    # V: one scale per channel over all tokens
+    vs = ops["v_chscale"].astype(np.float64)
+    assert np.allclose(vs, (np.abs(vf).max(0).astype(np.float32) / np.float32(448)), rtol=0, atol=0)
+    vrec = dec[ops["VcT"][:, :N].T] * vs[None, :]
+    assert np.all(np.abs(vrec - vf) <= _e4m3_err_bound(vf / vs[None, :]) * vs[None, :])
+
+
+def test_sage_attention_is_exact_softmax_on_its_dequantised_operands():
+    # with exact exponentials the row algorithm must equal plain softmax
+    # attention on Q^, K'^ (the smoothed keys) and V^ * channel scale
+    rng = np.random.default_rng(42)
+    N = 350
+    Q, K, V = _bits(rng, N), _bits(rng, N), _bits(rng, N)
+    ops = oracle.sage_quantize_head(Q, K, V)
+    dec = _e4m3_table()
+    sc = 1 / math.sqrt(128)
+    rows = np.arange(0, N, 11, dtype=np.int32)
+    got, _ = oracle.attention_head_sage(ops, N, sc, rows=rows, flags=oracle.EXACT_EXP)
+    q = dec[ops["Qq"][:N]] * ops["q_scale"][:N, None]
+    k = dec[ops["Kq"][:N]] * np.repeat(ops["k_scale"], 16)[:N, None]
+    v = dec[ops["VcT"][:, :N].T] * ops["v_chscale"][None, :].astype(np.float64)
+    s = q[rows] @ k.T * sc
+    p = np.exp(s - s.max(1, keepdims=True))
+    want = p @ v / p.sum(1, keepdims=True)
+    assert np.abs(got - want).max() < 1e-10
+
+
+def test_k_mean_smoothing_leaves_softmax_attention_unchanged():
+    # the identity the recipe relies on: q.(k - mu) = q.k - q.mu, a per-row shift
+    rng = np.random.default_rng(43)
+    q, k, v = rng.standard_normal((40, 128)), rng.standard_normal((90, 128)) + 3.0, rng.standard_normal((90, 128))
+    def att(kk):
+        s = q @ kk.T / math.sqrt(128)
+        p = np.exp(s - s.max(1, keepdims=True))
+        return p @ v / p.sum(1, keepdims=True)
+    assert np.abs(att(k) - att(k - k.mean(0))).max() < 1e-12
