@@ -66,6 +66,7 @@ struct AttnParams {
   unsigned long long wait_ns;
   float skip_log2;               // Skip Softmax: log2(lambda), -inf when off
   unsigned long long* skipped;   // optional count of skipped (query tile, key block) pairs
+  const float* v_chscale;        // SAGE operands: per-channel V scale [B*H][128]
 };
 
 
@@ -93,7 +94,10 @@ __device__ __forceinline__ uint32_t tf32_tile_off(int r, int k) {
 // 0 (no probability, zero row sum); a warp whose 32 rows all reject skips its
 // code pass (it stores zero codes), and when all four warps of a query tile do,
 // the MMA warp skips the tile's PV.
-template <bool SKIP>
+// SAGE: operands of the SAGE-style comparison recipe (vca_sage_quantize_qkv):
+// one Q scale per token, one K scale per 16 keys, V with per-channel scales
+// applied to the output and no block exponents or means (no mean restore).
+template <bool SKIP, bool SAGE>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -222,7 +226,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
             mma_mxf8_ts_w(tmem + 256 + t * 128, sft + 8 + 8 * k, dV + (uint64_t)(s * 1024 + 2 * k), id_pv, sft,
                           sft + 4, (j > 0 || k > 0) ? 1u : 0u);
         }
-        if (group_end) {
+        if (group_end && !SAGE) {
           ok = mbar_wait_warp(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220);
           if (!ok) break;
           tc_fence_after();
@@ -250,7 +254,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     }
     tc_commit_w(&bars.mma_done);
     if (SKIP && lane == 0 && p.skipped && nskip) atomicAdd(p.skipped, nskip);
-  } else if (warp == 2) {
+  } else if (warp == 2 && !SAGE) {
     // ------------------------------------------------------------ block means -> fp32 [d][8] tiles
     const uint16_t* vm = p.v_mean + (int64_t)bh * nb * 128;
     for (int g = 0; g < ngroups; ++g) {
@@ -278,7 +282,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const int qtile = pair * 2 + t;
     const bool qvalid = qtile < nb;
     const bool row_valid = qvalid && qtile * 128 + r < N;
-    const float sq = qvalid ? __ldg(p.q_scale + (int64_t)bh * nb + qtile) : 1.0f;
+    const float sq = !qvalid ? 1.0f
+                     : SAGE ? __ldg(p.q_scale + (int64_t)bh * Np + (int64_t)qtile * 128 + r)
+                            : __ldg(p.q_scale + (int64_t)bh * nb + qtile);
     const float cq = sq * p.c_base;
     const float kMagic = 12582912.0f;              // 1.5 * 2^23: adding it rounds to an integer
     uint8_t* sLt = sm + kOffL + t * 8192;
@@ -291,14 +297,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     bool ok = true;
     // the next tile's K scale and V exponent are loaded one tile ahead, off the
     // critical path of the score -> code computation
-    float ksc_next = __ldg(ksc);
-    int vex_next = __ldg(vex);
+    // SAGE: eight K scales per key block (one per 16 keys)
+    const float* ksc16 = p.k_scale + (int64_t)bh * (Np / 16);
+    float ksc_next = SAGE ? 0.0f : __ldg(ksc);
+    int vex_next = SAGE ? 0 : __ldg(vex);
+    float k8_next[8];
+    if (SAGE) {
+#pragma unroll
+      for (int g = 0; g < 8; ++g) k8_next[g] = __ldg(ksc16 + g);
+    }
     for (int j = 0; j < nkv; ++j) {
       const float ksc_j = ksc_next;
       const int vex_j = vex_next;
+      float k8[8];
+      if (SAGE) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g) k8[g] = k8_next[g];
+      }
       if (j + 1 < nkv) {
-        ksc_next = __ldg(ksc + j + 1);
-        vex_next = __ldg(vex + j + 1);
+        if (SAGE) {
+#pragma unroll
+          for (int g = 0; g < 8; ++g) k8_next[g] = __ldg(ksc16 + (j + 1) * 8 + g);
+        } else {
+          ksc_next = __ldg(ksc + j + 1);
+          vex_next = __ldg(vex + j + 1);
+        }
       }
       ok = mbar_wait_warp(&bars.s_full[t], j & 1, &abort_s, p.st, lim, 400 + t);
       if (!ok) break;
@@ -318,28 +341,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         for (int c = 0; c < 128; ++c)
           if (c >= valid) sv[c] = -INFINITY;
       }
-      // row maximum: four independent chains of 3-input max, chain q over the
-      // 32 scores sv[32q .. 32q+31]
-      float mq[4];
+      float mx = 0.0f, zmx = 0.0f;   // block maximum: raw score / in log2 units (SAGE)
+      float c8g[8];                   // SAGE: code multiplier of each 16-key group
+      if (!SAGE) {
+        // row maximum: four independent chains of 3-input max, chain q over the
+        // 32 scores sv[32q .. 32q+31]
+        float mq[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float m = sv[32 * q];
+        for (int q = 0; q < 4; ++q) {
+          float m = sv[32 * q];
 #pragma unroll
-        for (int i = 1; i < 31; i += 2) m = fmax3(m, sv[32 * q + i], sv[32 * q + i + 1]);
-        mq[q] = fmaxf(m, sv[32 * q + 31]);
+          for (int i = 1; i < 31; i += 2) m = fmax3(m, sv[32 * q + i], sv[32 * q + i + 1]);
+          mq[q] = fmaxf(m, sv[32 * q + 31]);
+        }
+        mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+      } else {
+        // one chain per 16-key group (its own K scale): z max = max_g(max s * cz_g)
+        zmx = -INFINITY;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          float m = sv[16 * g];
+#pragma unroll
+          for (int i = 1; i < 15; i += 2) m = fmax3(m, sv[16 * g + i], sv[16 * g + i + 1]);
+          m = fmaxf(m, sv[16 * g + 15]);
+          const float czg = cq * k8[g];
+          c8g[g] = 8.0f * czg;
+          zmx = fmaxf(zmx, m * czg);
+        }
       }
-      const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
       const float cz = cq * ksc_j;                 // z = s * cz (log2 domain)
       const float c8 = 8.0f * cz;
       bool rej = false;           // Skip Softmax: this row drops the block
       if (SKIP) {
-        const float zt = mx * cz;
+        const float zt = SAGE ? zmx : mx * cz;
         zrun = fmaxf(zrun, zt);
         // rows past the end of the sequence (padding of the last query tile)
         // vote to drop every block, so they never hold a whole-tile skip back
         rej = j > 0 && (!row_valid || zt - zrun < p.skip_log2);
       }
-      const int ntile = (int)ceilf(__fmaf_rn(mx, cz, -0.08125f));
+      const int ntile = (int)ceilf(SAGE ? zmx - 0.08125f : __fmaf_rn(mx, cz, -0.08125f));
       // (S_t(j) was committed after PV_t(j-1) and any mean MMA before it, so
       // those have completed: O_t may be rescaled and sL_t rewritten now)
       float rescale = 1.0f;       // O_t and the pending row sums are scaled by this
@@ -372,8 +412,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
         const int c = q * 4;
-        const float2 f01 = __ffma2_rn(make_float2(sv[c], sv[c + 1]), c8x2, baddx2);
-        const float2 f23 = __ffma2_rn(make_float2(sv[c + 2], sv[c + 3]), c8x2, baddx2);
+        const float c8q = SAGE ? (rej ? 0.0f : c8g[q >> 2]) : 0.0f;
+        const float2 cx = SAGE ? make_float2(c8q, c8q) : c8x2;
+        const float2 f01 = __ffma2_rn(make_float2(sv[c], sv[c + 1]), cx, baddx2);
+        const float2 f23 = __ffma2_rn(make_float2(sv[c + 2], sv[c + 3]), cx, baddx2);
         const uint32_t b0 = __float_as_uint(fmaxf(f01.x, kMagic)), b1 = __float_as_uint(fmaxf(f01.y, kMagic));
         const uint32_t b2 = __float_as_uint(fmaxf(f23.x, kMagic)), b3 = __float_as_uint(fmaxf(f23.y, kMagic));
         lsa = __fadd2_rn(lsa, make_float2(__uint_as_float(b0 << 20), __uint_as_float(b1 << 20)));
@@ -385,7 +427,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       const float lsum = (lsa.x + lsa.y) + (lsb.x + lsb.y);
       const float l = lsum * 0x1p120f;
       // block row sum -> L tile (hi part exact in TF32, lo the remainder)
-      {
+      if (!SAGE) {
         const int kk = j % kGroup;
         const float hi = __uint_as_float(__float_as_uint(l) & 0xFFFFE000u);
         const float lo = l - hi;
@@ -411,7 +453,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
           for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * rescale);
           VCA_TMEM_ST32(tO + c0, o);
         }
-        for (int kk = 0; kk < (j % kGroup); ++kk) {
+        for (int kk = 0; kk < (SAGE ? 0 : j % kGroup); ++kk) {
           float* hi = reinterpret_cast<float*>(sLt + tf32_tile_off(r, kk));
           float* lo = reinterpret_cast<float*>(sLt + 4096 + tf32_tile_off(r, kk));
           *hi *= rescale;
@@ -451,8 +493,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(o[2 * c]) * inv,
-                                                     __uint_as_float(o[2 * c + 1]) * inv);
+            float o0 = __uint_as_float(o[2 * c]) * inv, o1 = __uint_as_float(o[2 * c + 1]) * inv;
+            if (SAGE) {
+              o0 *= __ldg(p.v_chscale + bh * 128 + c0 + 2 * c);
+              o1 *= __ldg(p.v_chscale + bh * 128 + c0 + 2 * c + 1);
+            }
+            __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
             pk[c] = *reinterpret_cast<uint32_t*>(&h);
           }
           uint4* dst = reinterpret_cast<uint4*>(orow + c0);
@@ -487,7 +533,8 @@ static int attention_launch(const char* fn, const uint8_t* Qq, const float* q_sc
                             const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
                             const vca_bf16* v_mean, int B, int H, int N, int d, float softmax_scale,
                             vca_bf16* O, float* lse, void* ws, size_t ws_bytes, float skip_lambda,
-                            unsigned long long* skipped, vca_stream_t stream) {
+                            unsigned long long* skipped, const float* v_chscale, vca_stream_t stream) {
+  const bool sage = v_chscale != nullptr;   // SAGE operands: no V exponents or means
   if (d != VCA_HEAD_DIM) return fail(VCA_ERR_UNSUPPORTED, "%s: d must be 128", fn);
   if (B < 1 || H < 1 || N < 1 || (int64_t)B * H > 65535)
     return fail(VCA_ERR_INVALID, "%s: bad shape B=%d H=%d N=%d", fn, B, H, N);
@@ -495,9 +542,10 @@ static int attention_launch(const char* fn, const uint8_t* Qq, const float* q_sc
   const int64_t Np = (int64_t)nb * 128;
   if ((int64_t)B * H * Np > INT32_MAX || Np > INT32_MAX / 2)
     return fail(VCA_ERR_UNSUPPORTED, "%s: B*H*Np exceeds the 2^31 row limit", fn);
-  const void* ptrs[] = {Qq, q_scale, Kq, k_scale, VrT, v_exp, v_mean, O};
+  const void* ptrs[] = {Qq, q_scale, Kq, k_scale, VrT, O};
   for (const void* q : ptrs)
     if (!q) return fail(VCA_ERR_INVALID, "%s: null pointer", fn);
+  if (!sage && (!v_exp || !v_mean)) return fail(VCA_ERR_INVALID, "%s: null pointer", fn);
   const void* al[] = {Qq, Kq, VrT, O};
   for (const void* q : al)
     if (!aligned16(q)) return fail(VCA_ERR_INVALID, "%s: tensors must be 16-byte aligned", fn);
@@ -532,7 +580,9 @@ static int attention_launch(const char* fn, const uint8_t* Qq, const float* q_sc
   const bool skip = skip_lambda > 0.0f;
   prm.skip_log2 = skip ? (float)log2((double)skip_lambda) : -INFINITY;
   prm.skipped = skipped;
-  auto kern = skip ? attn_fp8_kernel<true> : attn_fp8_kernel<false>;
+  prm.v_chscale = v_chscale;
+  if (skip && sage) return fail(VCA_ERR_UNSUPPORTED, "%s: Skip Softmax on SAGE operands is not built", fn);
+  auto kern = skip ? attn_fp8_kernel<true, false> : sage ? attn_fp8_kernel<false, true> : attn_fp8_kernel<false, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc) != cudaSuccess)
     return fail(VCA_ERR_CUDA, "%s: cannot set shared-memory size", fn);
   dim3 grid((nb + 1) / 2, (unsigned)BH);
@@ -546,7 +596,7 @@ extern "C" int vca_attention_fwd(const uint8_t* Qq, const float* q_scale, const 
                                  float softmax_scale, vca_bf16* O, float* lse, void* ws,
                                  size_t ws_bytes, vca_stream_t stream) {
   return attention_launch("vca_attention_fwd", Qq, q_scale, Kq, k_scale, VrT, v_exp, v_mean, B, H, N, d,
-                          softmax_scale, O, lse, ws, ws_bytes, 0.0f, nullptr, stream);
+                          softmax_scale, O, lse, ws, ws_bytes, 0.0f, nullptr, nullptr, stream);
 }
 
 extern "C" int vca_attention_fwd_skip(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
@@ -556,5 +606,14 @@ extern "C" int vca_attention_fwd_skip(const uint8_t* Qq, const float* q_scale, c
                                       unsigned long long* skipped_tiles, void* ws, size_t ws_bytes,
                                       vca_stream_t stream) {
   return attention_launch("vca_attention_fwd_skip", Qq, q_scale, Kq, k_scale, VrT, v_exp, v_mean, B, H, N, d,
-                          softmax_scale, O, lse, ws, ws_bytes, skip_lambda, skipped_tiles, stream);
+                          softmax_scale, O, lse, ws, ws_bytes, skip_lambda, skipped_tiles, nullptr, stream);
+}
+
+extern "C" int vca_attention_fwd_sage(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                                      const float* k_scale, const uint8_t* VcT, const float* v_chscale, int B,
+                                      int H, int N, int d, float softmax_scale, vca_bf16* O, float* lse, void* ws,
+                                      size_t ws_bytes, vca_stream_t stream) {
+  if (!v_chscale) return fail(VCA_ERR_INVALID, "vca_attention_fwd_sage: null pointer");
+  return attention_launch("vca_attention_fwd_sage", Qq, q_scale, Kq, k_scale, VcT, nullptr, nullptr, B, H, N, d,
+                          softmax_scale, O, lse, ws, ws_bytes, 0.0f, nullptr, v_chscale, stream);
 }

@@ -332,6 +332,43 @@ __host__ __device__ constexpr uint32_t instr_desc_mx(uint32_t afmt, uint32_t bfm
 __device__ __forceinline__ uint32_t f32_bits(float f) { return __float_as_uint(f); }
 __device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
 
+// bf16 halves of a 32-bit word as fp32 (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Round a double to bf16, nearest-even, in one step on the integer bits.
+__device__ __forceinline__ uint16_t double_to_bf16_rne(double x) {
+  unsigned long long b = (unsigned long long)__double_as_longlong(x);
+  unsigned long long sign = b >> 63;
+  unsigned long long a = b & 0x7FFFFFFFFFFFFFFFull;
+  if (a == 0) return (uint16_t)(sign << 15);
+  int e = (int)(a >> 52) - 1023;
+  if (e >= -126) {
+    // keep 7 fraction bits of the double's 52: round at bit 45
+    unsigned long long lsb = (a >> 45) & 1ull;
+    unsigned long long r = (a + 0x00000FFFFFFFFFFFull + lsb) >> 45;   // exponent | 7-bit fraction
+    int e2 = (int)(r >> 7) - 1023;
+    if (e2 > 127) return (uint16_t)((sign << 15) | 0x7F80u);
+    return (uint16_t)((sign << 15) | ((unsigned)(e2 + 127) << 7) | (unsigned)(r & 0x7F));
+  }
+  // bf16 subnormal range: value = m * 2^-133, m in [0, 128]
+  double m = rint(x < 0 ? -x * 0x1p133 : x * 0x1p133);
+  return (uint16_t)((sign << 15) | (unsigned)m);
+}
+
+// Exact split of llrint(v * 2^24) for |v| < 2^20 (at most 45 bits) into
+// hi * 2^22 + lo with |hi|, |lo| < 2^22, using float operations only: f = v * 2^24
+// is exact, hi = trunc(f / 2^22), lo = rne(f - hi * 2^22) (the only rounding, the
+// same as llrint's); each becomes an integer through the magic-number add.
+__device__ __forceinline__ void fix24_split(float v, int& hi, int& lo) {
+  const float kMagic = 12582912.0f;   // 1.5 * 2^23
+  const float f = v * 16777216.0f;
+  const float hf = truncf(f * 2.384185791015625e-07f);     // f / 2^22, truncated
+  const float lf = __fmaf_rn(hf, -4194304.0f, f);         // exact remainder
+  hi = (int)(__float_as_uint(hf + kMagic) - 0x4B400000u);
+  lo = (int)(__float_as_uint(lf + kMagic) - 0x4B400000u);
+}
+
 // Two fp32 -> two E4M3 bytes, round-to-nearest-even, saturating (hardware cvt).
 // Result: low byte = e4m3(lo), next byte = e4m3(hi).
 __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {

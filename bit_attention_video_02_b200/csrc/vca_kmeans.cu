@@ -171,14 +171,6 @@ __global__ void __launch_bounds__(kAssignThreads) km_assign_kernel(const uint16_
 // addition is exact and order-free: the sums are exact whatever the order.
 constexpr int kSegTok = 256;   // sorted positions per warp
 constexpr int kSegWarps = 8;
-__device__ __forceinline__ void fix24_split(float v, int& hi, int& lo) {
-  const float kMagic = 12582912.0f;   // 1.5 * 2^23
-  const float f = v * 16777216.0f;
-  const float hf = truncf(f * 2.384185791015625e-07f);     // f / 2^22, truncated
-  const float lf = __fmaf_rn(hf, -4194304.0f, f);         // exact remainder
-  hi = (int)(__float_as_uint(hf + kMagic) - 0x4B400000u);
-  lo = (int)(__float_as_uint(lf + kMagic) - 0x4B400000u);
-}
 __global__ void __launch_bounds__(kSegWarps * 32) km_accum_kernel(const uint16_t* __restrict__ V,
                                                                  const int32_t* __restrict__ perm,
                                                                  const int* __restrict__ cstart,

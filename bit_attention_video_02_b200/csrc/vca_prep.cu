@@ -39,29 +39,6 @@ struct PrepArgs {
   int tensor_base;   // blockIdx.y + tensor_base: 0 = Q, 1 = K, 2 = V
 };
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// Round a double to bf16, nearest-even, in one step on the integer bits.
-__device__ __forceinline__ uint16_t double_to_bf16_rne(double x) {
-  unsigned long long b = (unsigned long long)__double_as_longlong(x);
-  unsigned long long sign = b >> 63;
-  unsigned long long a = b & 0x7FFFFFFFFFFFFFFFull;
-  if (a == 0) return (uint16_t)(sign << 15);
-  int e = (int)(a >> 52) - 1023;
-  if (e >= -126) {
-    // keep 7 fraction bits of the double's 52: round at bit 45
-    unsigned long long lsb = (a >> 45) & 1ull;
-    unsigned long long r = (a + 0x00000FFFFFFFFFFFull + lsb) >> 45;   // exponent | 7-bit fraction
-    int e2 = (int)(r >> 7) - 1023;
-    if (e2 > 127) return (uint16_t)((sign << 15) | 0x7F80u);
-    return (uint16_t)((sign << 15) | ((unsigned)(e2 + 127) << 7) | (unsigned)(r & 0x7F));
-  }
-  // bf16 subnormal range: value = m * 2^-133, m in [0, 128]
-  double m = rint(x < 0 ? -x * 0x1p133 : x * 0x1p133);
-  return (uint16_t)((sign << 15) | (unsigned)m);
-}
-
 // Smallest e with amax <= 448 * 2^e (0 for amax == 0), clamped to [-127, 127].
 // amax = (1 + f) 2^(E-127) = ((1+f)/2) 2^(E-126); 448 = 0.875 2^9.
 __device__ __forceinline__ int v_exponent(float amax) {

@@ -34,6 +34,7 @@ EXPORTED = [
     "vca_attention_workspace_size", "vca_attention_fwd",
     "vca_bf16_attention_workspace_size", "vca_bf16_attention_fwd", "vca_schedule_regroup",
     "vca_attention_fwd_skip", "vca_vc_attention_host_buffer_size", "vca_vc_attention_host",
+    "vca_sage_quantize_workspace_size", "vca_sage_quantize_qkv", "vca_attention_fwd_sage",
 ]
 
 
@@ -73,6 +74,10 @@ def lib() -> ctypes.CDLL:
         L.vca_bf16_attention_fwd.argtypes = [vp, vp, vp, i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
         L.vca_schedule_regroup.argtypes = [i32, i32, i32, f32]
         L.vca_attention_fwd_skip.argtypes = [vp] * 7 + [i32, i32, i32, i32, f32, f32, vp, vp, vp, vp, sz, vp]
+        L.vca_sage_quantize_workspace_size.restype = sz
+        L.vca_sage_quantize_workspace_size.argtypes = [i32, i32, i32]
+        L.vca_sage_quantize_qkv.argtypes = [vp, vp, vp] + [i32] * 4 + [vp] * 7 + [vp, sz, vp]
+        L.vca_attention_fwd_sage.argtypes = [vp] * 6 + [i32] * 4 + [f32, vp, vp, vp, sz, vp]
         L.vca_vc_attention_host_buffer_size.restype = sz
         L.vca_vc_attention_host_buffer_size.argtypes = [i32] * 6
         L.vca_vc_attention_host.argtypes = [vp, vp, vp] + [i32] * 6 + [f32, vp, i32, vp, sz, vp]
@@ -80,7 +85,8 @@ def lib() -> ctypes.CDLL:
                    "vca_e4m3_encode", "vca_cluster_permute", "vca_cluster_permute_noalloc",
                    "vca_smooth_quantize_qkv",
                    "vca_attention_fwd", "vca_bf16_attention_fwd", "vca_schedule_regroup",
-                   "vca_attention_fwd_skip", "vca_vc_attention_host"):
+                   "vca_attention_fwd_skip", "vca_vc_attention_host", "vca_sage_quantize_qkv",
+                   "vca_attention_fwd_sage"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -339,3 +345,43 @@ def vc_attention_host(Q, K, V, k: int = 32, iters: int = 3, softmax_scale=None, 
                                            heads_per_chunk, ctypes.c_void_p(buf.data_ptr()), need,
                                            _stream(stream)))
     return O
+
+
+def sage_quantize(Q, K, V, ws: Workspace | None = None, stream=None) -> dict:
+    """vca_sage_quantize_qkv: the SAGE-style comparison quantisation."""
+    B, H, N, d = _bhnd(Q)
+    dev = Q.device
+    nb = (N + 127) // 128
+    Np = nb * 128
+    out = dict(Qq=torch.empty(B, H, Np, d, dtype=torch.uint8, device=dev),
+               q_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
+               Kq=torch.empty(B, H, Np, d, dtype=torch.uint8, device=dev),
+               k_scale=torch.empty(B, H, Np // 16, dtype=torch.float32, device=dev),
+               VcT=torch.empty(B, H, d, Np, dtype=torch.uint8, device=dev),
+               v_chscale=torch.empty(B, H, d, dtype=torch.float32, device=dev),
+               k_mean=torch.empty(B, H, d, dtype=torch.bfloat16, device=dev))
+    need = lib().vca_sage_quantize_workspace_size(B, H, N)
+    ws = (ws or Workspace(need, dev)).ensure(need)
+    _check(lib().vca_sage_quantize_qkv(
+        _ptr(Q), _ptr(K), _ptr(V), B, H, N, d, _ptr(out["Qq"]), _ptr(out["q_scale"]), _ptr(out["Kq"]),
+        _ptr(out["k_scale"]), _ptr(out["VcT"]), _ptr(out["v_chscale"]), _ptr(out["k_mean"]), ws.ptr, ws.nbytes,
+        _stream(stream)))
+    return out
+
+
+def attention_fwd_sage(ops: dict, N: int, softmax_scale: float | None = None, O=None, lse=None,
+                       want_lse: bool = False, ws: Workspace | None = None, stream=None):
+    """vca_attention_fwd_sage: FP8 attention on SAGE-style operands."""
+    B, H, Np, d = ops["Qq"].shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dev = ops["Qq"].device
+    if O is None:
+        O = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    need = lib().vca_attention_workspace_size(B, H, N)
+    ws = (ws or Workspace(need, dev)).ensure(need)
+    _check(lib().vca_attention_fwd_sage(
+        _ptr(ops["Qq"]), _ptr(ops["q_scale"]), _ptr(ops["Kq"]), _ptr(ops["k_scale"]), _ptr(ops["VcT"]),
+        _ptr(ops["v_chscale"]), B, H, N, d, scale, _ptr(O), _ptr(lse), ws.ptr, ws.nbytes, _stream(stream)))
+    return (O, lse) if want_lse else O

@@ -256,6 +256,34 @@ int vca_vc_attention_host(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* 
                           int d, int k, int iters, float softmax_scale, vca_bf16* O, int heads_per_chunk,
                           void* dev_buf, size_t dev_bytes, vca_stream_t stream);
 
+/* SAGE-style comparison recipe on the same harness ([TRT-blog], section
+ * "Quantized Attention": q_block_size 1, k_block_size 16, v_block_size 1, FP8 V,
+ * following the SageAttention2 line of work, whose K smoothing is applied).
+ * Per (b, h), no reordering and no block means:
+ *   k_mean[c]   = bf16(exact mean of K[:, c] over the N tokens)
+ *   Qq, q_scale one fp32 scale per token: max|x| / 448, codes e4m3(x * 448/max|x|)
+ *   Kq, k_scale K' = K - k_mean (fp32), one scale per 16 tokens, same formula
+ *   VcT, v_chscale  one scale per channel over all N tokens, same formula;
+ *               VcT is channel-major like VrT
+ * An all-zero group has scale 1 and codes 0; padding rows and keys are 0.
+ * Shapes: Qq, Kq [B][H][Np][d] u8; q_scale [B][H][Np] f32; k_scale
+ * [B][H][Np/16] f32; VcT [B][H][d][Np] u8; v_chscale [B][H][d] f32; k_mean
+ * [B][H][d] bf16.  |K| < 2^20 (exact fixed-point mean), finite inputs. */
+size_t vca_sage_quantize_workspace_size(int B, int H, int N);
+int vca_sage_quantize_qkv(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V, int B, int H, int N, int d,
+                          uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale, uint8_t* VcT,
+                          float* v_chscale, vca_bf16* k_mean, void* ws, size_t ws_bytes, vca_stream_t stream);
+
+/* The FP8 attention of vca_attention_fwd (ExpCast codes, online reference,
+ * tcgen05 MMAs) on SAGE-style operands: z uses the token's Q scale and the
+ * 16-key group's K scale; PV has no block exponent and there is no mean
+ * restore; output channel c is multiplied by v_chscale[c] after the
+ * normalisation.  Workspace as vca_attention_fwd. */
+int vca_attention_fwd_sage(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq, const float* k_scale,
+                           const uint8_t* VcT, const float* v_chscale, int B, int H, int N, int d,
+                           float softmax_scale, vca_bf16* O, float* lse, void* ws, size_t ws_bytes,
+                           vca_stream_t stream);
+
 /* In-repo BF16 comparator: exact-softmax flash attention (online softmax with
  * exp2), tcgen05 BF16 MMAs with fp32 accumulation in tensor memory.
  *   Q, K, V, O [B][H][N][d] bf16; lse [B][H][N] fp32 natural log (nullable). */

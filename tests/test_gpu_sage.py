@@ -1,0 +1,77 @@
+"""SAGE-style comparison recipe ("Accelerating Video Generation with GEMM
+Quantization, Attention Quantization and Skip Softmax Attention in
+TensorRT-LLM", section "Quantized Attention") on the GPU: the quantisation bit
+for bit against the oracle, the FP8 attention on its operands within the
+attention tolerance, and its fidelity beside V-Smooth's on the same inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_attention_video_02_b200 import vca
+from bit_attention_video_02_b200 import workloads as W
+from helpers import bf16_to_f64, bits, cosine, rel_l2, sample_rows
+
+pytestmark = pytest.mark.gpu
+CASES = [(1, None, None), (2, 2, 1500), (3, 2, 1000), (5, 1, 700)]
+
+
+def _ids(c):
+    return f"cfg{c[0]}" + (f"_H{c[1]}_N{c[2]}" if c[1] else "")
+
+
+@pytest.mark.parametrize("case", CASES, ids=_ids)
+def test_sage_quantisation_bit_exact(case):
+    cid, H, N = case
+    w = W.WORKLOADS[cid] if H is None else W.shrink(W.WORKLOADS[cid], H=H, N=N)
+    Q, K, V = W.make_qkv(w, "cuda")
+    ops = vca.sage_quantize(Q, K, V)
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        ref = oracle.sage_quantize_head(bits(Q[0, h]), bits(K[0, h]), bits(V[0, h]))
+        for key in ("Qq", "Kq", "VcT", "q_scale", "k_scale", "v_chscale"):
+            got = ops[key][0, h].cpu().numpy()
+            assert np.array_equal(got, ref[key]), (key, h)
+        assert np.array_equal(bits(ops["k_mean"][0, h]), ref["k_mean"])
+
+
+@pytest.mark.parametrize("case", CASES, ids=_ids)
+def test_sage_attention_matches_oracle(case):
+    cid, H, N = case
+    w = W.WORKLOADS[cid] if H is None else W.shrink(W.WORKLOADS[cid], H=H, N=N)
+    Q, K, V = W.make_qkv(w, "cuda")
+    scale = 1.0 / math.sqrt(w.d)
+    ops = vca.sage_quantize(Q, K, V)
+    O = vca.attention_fwd_sage(ops, w.N, scale)
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        ref = {k: v[0, h].cpu().numpy() for k, v in ops.items() if k != "k_mean"}
+        rows = sample_rows(w.N, 200, 900 + h)
+        o_ref, _ = oracle.attention_head_sage(ref, w.N, scale, rows=rows)
+        g = bf16_to_f64(O[0, h])[rows]
+        ex = oracle.exact_attention_head(bits(Q[0, h]), bits(K[0, h]), bits(V[0, h]), scale, rows=rows)
+        print(dict(case=_ids(case), head=h, rel_l2=rel_l2(g, o_ref), cos=cosine(g, ex)))
+        assert rel_l2(g, o_ref) <= 1e-2
+        assert cosine(g, ex) >= 0.99
+
+
+@pytest.mark.parametrize("cid", [2, 3])
+def test_fidelity_vsmooth_beside_sage(cid):
+    # same inputs, both recipes, error against exact attention; reported, and
+    # both must stay inside the fidelity bar
+    w = W.shrink(W.WORKLOADS[cid], H=2, N=3000)
+    Q, K, V = W.make_qkv(w, "cuda")
+    scale = 1.0 / math.sqrt(w.d)
+    O_vc = vca.vc_attention(Q, K, V, k=w.k, iters=3)
+    O_sg = vca.attention_fwd_sage(vca.sage_quantize(Q, K, V), w.N, scale)
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        rows = sample_rows(w.N, 256, 50 + h)
+        ex = oracle.exact_attention_head(bits(Q[0, h]), bits(K[0, h]), bits(V[0, h]), scale, rows=rows)
+        e_vc = rel_l2(bf16_to_f64(O_vc[0, h])[rows], ex)
+        e_sg = rel_l2(bf16_to_f64(O_sg[0, h])[rows], ex)
+        print(dict(cfg=cid, head=h, rel_l2_vsmooth=e_vc, rel_l2_sage=e_sg))
+        assert cosine(bf16_to_f64(O_vc[0, h])[rows], ex) >= 0.99
+        assert cosine(bf16_to_f64(O_sg[0, h])[rows], ex) >= 0.99
