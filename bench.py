@@ -267,6 +267,38 @@ def run_ours(args, world, rank, local):
                                       "what": "workload Q, V; K x12 on even key blocks; identity order"}}
         ws.check()
 
+    # ---- SAGE-style comparison recipe on the same inputs: prep and attention
+    # time, and the fidelity of both recipes against the exact-softmax BF16
+    # kernel's output (over the whole layer, on the GPU)
+    sage = None
+    if not args.no_sage:
+        sops = vca.sage_quantize(Q, K, V, ws=ws)
+        O_sg = vca.attention_fwd_sage(sops, N, scale, ws=ws)
+        g0, g1, g2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        torch.cuda.synchronize()
+        g0.record(stream)
+        for _ in range(3):
+            vca.sage_quantize(Q, K, V, ws=ws)
+        g1.record(stream)
+        for _ in range(3):
+            vca.attention_fwd_sage(sops, N, scale, O=O_sg, ws=ws)
+        g2.record(stream)
+        torch.cuda.synchronize()
+        O_vc = vca.attention_fwd(ops, N, scale, ws=ws)
+        O_ex = vca.bf16_attention_fwd(Q, K, V, scale, ws=ws)
+        torch.cuda.synchronize()
+
+        def fid(a):
+            a, b = a.float(), O_ex.float()
+            return {"rel_l2": round((torch.linalg.vector_norm(a - b) / torch.linalg.vector_norm(b)).item(), 5),
+                    "cosine": round((torch.sum(a * b) / (torch.linalg.vector_norm(a) *
+                                                         torch.linalg.vector_norm(b))).item(), 6)}
+
+        sage = {"prep_ms": round(g0.elapsed_time(g1) / 3, 3), "attn_ms": round(g1.elapsed_time(g2) / 3, 3),
+                "fidelity_vs_bf16_exact_softmax": {"v_smooth": fid(O_vc), "sage": fid(O_sg)}}
+        del sops, O_sg, O_vc, O_ex
+        ws.check()
+
     # ---- end to end through the C ABI with host buffers: vca_vc_attention_host
     # takes page-locked host Q, K, V and returns the host O, its copies
     # overlapped with the kernels (each step copies all inputs in and O out)
@@ -331,6 +363,7 @@ def run_ours(args, world, rank, local):
         "quant_only_ms": round(quant_ms, 3),
         "bf16_attn_ms": round(bf16_ms, 3) if bf16_ms else None,
         "skip_softmax": skip,
+        "sage_comparison": sage,
         "fp8_over_bf16": round(bf16_ms / (t_attn * 1e3), 3) if bf16_ms else None,
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp8_peak_sust, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / fp8_peak_sust, 4), "traffic": traffic,
@@ -467,6 +500,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-bf16", action="store_true")
     ap.add_argument("--no-skip", action="store_true")
+    ap.add_argument("--no-sage", action="store_true")
     ap.add_argument("--skip-lambda", type=float, default=2.0 ** -6)
     args = ap.parse_args()
     world, rank, local = dist_setup(args)
