@@ -118,50 +118,55 @@ __global__ void __launch_bounds__(kBfThreads, 1) attn_bf16_kernel(const __grid_c
           mbar_wait_bounded(&bars.kv_full[j % kBfStages], (j / kBfStages) & 1, &never_s, nullptr, lim, 101);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t id_qk = instr_desc(kFmtBF16, kFmtBF16, 128, 128, 0, 0);
-      const uint32_t id_pv = instr_desc(kFmtBF16, kFmtBF16, 128, 128, 0, 1);
-      const uint32_t sQ = smem_u32(sm + kBfOffQ), sK = smem_u32(sm + kBfOffK), sV = smem_u32(sm + kBfOffV);
-      bool ok = mbar_wait_bounded(&bars.q_full, 0, &abort_s, p.st, lim, 200);
-      ok = ok && mbar_wait_bounded(&bars.kv_full[0], 0, &abort_s, p.st, lim, 201);
-      auto issue_qk = [&](int t, int s) {
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-          mma_bf16_ss(tmem + t * 128, smem_desc(sQ + t * 32768 + off, 16, 1024, kLayoutSW128),
-                      smem_desc(sK + s * 32768 + off, 16, 1024, kLayoutSW128), id_qk, k > 0);
-        }
-        tc_commit(&bars.s_full[t]);
-      };
-      if (ok) {
-        tc_fence_after();
-        issue_qk(0, 0);
-        issue_qk(1, 0);
+    // the whole warp runs the issue loop (warp-uniform descriptors advanced by
+    // constants); one elected lane issues each tcgen05 instruction
+    const uint32_t id_qk = instr_desc(kFmtBF16, kFmtBF16, 128, 128, 0, 0);
+    const uint32_t id_pv = instr_desc(kFmtBF16, kFmtBF16, 128, 128, 0, 1);
+    // descriptor start addresses count 16-byte units
+    const uint64_t dQ = smem_desc(smem_u32(sm + kBfOffQ), 16, 1024, kLayoutSW128);
+    const uint64_t dK = smem_desc(smem_u32(sm + kBfOffK), 16, 1024, kLayoutSW128);
+    const uint64_t dV = smem_desc(smem_u32(sm + kBfOffV), 16384, 1024, kLayoutSW128);
+    bool ok = mbar_wait_warp(&bars.q_full, 0, &abort_s, p.st, lim, 200);
+    ok = ok && mbar_wait_warp(&bars.kv_full[0], 0, &abort_s, p.st, lim, 201);
+    auto issue_qk = [&](int t, int s) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint64_t off = (uint64_t)((k >> 2) * 1024 + (k & 3) * 2);   // (k/4)*16 KB + (k%4)*32 B
+        mma_bf16_ss_w(tmem + t * 128, dQ + (uint64_t)(t * 2048) + off, dK + (uint64_t)(s * 2048) + off, id_qk,
+                      k > 0);
       }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % kBfStages;
-        for (int t = 0; t < 2 && ok; ++t) {
-          ok = mbar_wait_bounded(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t);
-          if (!ok) break;
-          tc_fence_after();
-          for (int k = 0; k < 8; ++k)
-            mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + 8 * k,
-                        smem_desc(sV + s * 32768 + k * 2048, 16384, 1024, kLayoutSW128), id_pv,
-                        (j > 0 || k > 0) ? 1u : 0u);
-          tc_commit(&bars.o_done[t]);
-          if (t == 1) tc_commit(&bars.kv_empty[s]);
-          if (j + 1 < nkv) {
-            const int s1 = (j + 1) % kBfStages;
-            if (t == 0) {
-              ok = mbar_wait_bounded(&bars.kv_full[s1], ((j + 1) / kBfStages) & 1, &abort_s, p.st, lim, 230);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            issue_qk(t, s1);
-          }
-        }
-      }
-      tc_commit(&bars.mma_done);
+      tc_commit_w(&bars.s_full[t]);
+    };
+    if (ok) {
+      tc_fence_after();
+      issue_qk(0, 0);
+      issue_qk(1, 0);
     }
+    for (int j = 0; ok && j < nkv; ++j) {
+      const int s = j % kBfStages;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        ok = mbar_wait_warp(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          mma_bf16_ts_w(tmem + 256 + t * 128, tmem + t * 128 + 8 * k, dV + (uint64_t)(s * 2048 + k * 128), id_pv,
+                        (j > 0 || k > 0) ? 1u : 0u);
+        tc_commit_w(&bars.o_done[t]);
+        if (t == 1) tc_commit_w(&bars.kv_empty[s]);
+        if (j + 1 < nkv) {
+          const int s1 = (j + 1) % kBfStages;
+          if (t == 0) {
+            ok = mbar_wait_warp(&bars.kv_full[s1], ((j + 1) / kBfStages) & 1, &abort_s, p.st, lim, 230);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          issue_qk(t, s1);
+        }
+      }
+    }
+    tc_commit_w(&bars.mma_done);
   } else if (warp >= 4) {
     const int t = (warp >> 2) - 1;
     const int r = threadIdx.x & 127;
