@@ -143,72 +143,7 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-// Arrives once on `bar` when every tcgen05 operation this thread issued before
-// it has completed.
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
 
-// D[tmem] (+)= A[smem] * B[smem]^T, 8-bit E4M3 operands (kind::f8f6f4).
-__device__ __forceinline__ void mma_f8_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                          uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum));
-}
-// Same with UE8M0 block scales read from TMEM (kind::mxf8f6f4.block_scale).
-__device__ __forceinline__ void mma_mxf8_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                            uint32_t sfa, uint32_t sfb, uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
-          d),
-      "l"(a), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accum));
-}
-// Same, with A (the probabilities) read from tensor memory.
-__device__ __forceinline__ void mma_mxf8_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                            uint32_t sfa, uint32_t sfb, uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %6, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], [%1], %2, %3, [%4], [%5], p;\n\t}" ::"r"(
-          d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accum));
-}
-// TF32 operands (kind::tf32).
-__device__ __forceinline__ void mma_tf32_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                            uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum));
-}
-// BF16 operands, both from shared memory (kind::f16).
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                            uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum));
-}
-// BF16, A from tensor memory (kind::f16).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d, uint32_t a_tmem, uint64_t b,
-                                            uint32_t idesc, uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum));
-}
-// E4M3, A from tensor memory (kind::f8f6f4).
-__device__ __forceinline__ void mma_f8_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                          uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum));
-}
 
 // Warp-issued forms: the whole converged warp runs the issue loop in lockstep
 // (so descriptors and addresses stay warp-uniform and cost one set of uniform
@@ -290,10 +225,6 @@ __device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),      \
       "r"(r[15]))
 
-__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]),
-               "r"(r[1]), "r"(r[2]), "r"(r[3]));
-}
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
                    taddr),
@@ -343,8 +274,6 @@ __host__ __device__ constexpr uint32_t instr_desc_mx(uint32_t afmt, uint32_t bfm
 }
 
 // ---------------------------------------------------------------- numerics
-__device__ __forceinline__ uint32_t f32_bits(float f) { return __float_as_uint(f); }
-__device__ __forceinline__ float bits_f32(uint32_t u) { return __uint_as_float(u); }
 
 // bf16 halves of a 32-bit word as fp32 (exact).
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -391,19 +320,7 @@ __device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
   return r;
 }
 
-// fp32 fused multiply-add with the result clamped to [0, 1] (NaN -> 0)
-__device__ __forceinline__ float fma_sat(float a, float b, float c) {
-  float d;
-  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
 
-// x << 20 written as an integer multiply-add (issued on the FMA pipe)
-__device__ __forceinline__ uint32_t shl20_mad(uint32_t x) {
-  uint32_t d;
-  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(x), "r"(1u << 20), "r"(0u));
-  return d;
-}
 
 // max of three fp32 values in one instruction
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
