@@ -10,6 +10,7 @@
 // vca_smooth_quantize_qkv and vca_attention_fwd, so the result is the same, bit
 // for bit, as running the three calls on the whole layer.
 #include <mutex>
+#include <vector>
 
 #include "vca_host.h"
 
@@ -80,27 +81,30 @@ int get_streams(Streams* out) {
   return VCA_OK;
 }
 
-// Chunk c covers units [chunk_start(c), chunk_start(c + 1)).  The first and the
-// last chunk hold one unit each (with at least three units): the first chunk's
-// input copy and the last chunk's output copy are the only transfers nothing
-// overlaps, so they are kept small; the chunks between hold `u` units.
-int chunk_count(int units, int u) {
-  if (units < 3) return units;
-  return 2 + (units - 2 + u - 1) / u;
-}
-int chunk_start(int c, int units, int u) {
-  if (units < 3) return c;
-  if (c == 0) return 0;
-  const int n = chunk_count(units, u);
-  if (c >= n) return units;
-  if (c == n - 1) return units - 1;
-  const int s = 1 + (c - 1) * u;
-  return s < units - 1 ? s : units - 1;
+// Chunk boundaries: sizes double from one unit up to `u` (1, 2, 4, ..., u, u, ...)
+// and the last chunk holds one unit.  The first chunk's input copy and the last
+// chunk's output copy are the only transfers nothing overlaps, so they are kept
+// small; doubling lets each chunk's input copy fit under the previous chunk's
+// compute while the pipeline fills.  starts[i] is the first unit of chunk i,
+// starts.back() == units.
+std::vector<int> chunk_starts(int units, int u) {
+  std::vector<int> starts;
+  int pos = 0, size = 1;
+  while (pos < units) {
+    const int remaining = units - pos;
+    int take = size < remaining ? size : remaining;
+    if (take == remaining && remaining > 1) take = remaining - 1;   // the last unit goes alone
+    starts.push_back(pos);
+    pos += take;
+    size = 2 * size < u ? 2 * size : u;
+  }
+  starts.push_back(units);
+  return starts;
 }
 
 int units_per_chunk(int units, int heads_per_chunk) {
   if (heads_per_chunk > 0) return heads_per_chunk < units ? heads_per_chunk : units;
-  const int u = (units + 7) / 8;   // about eight chunks
+  const int u = (units + 4) / 5;   // about five chunks at full size, after the doubling ramp
   return u < 1 ? 1 : u;
 }
 
@@ -145,12 +149,13 @@ extern "C" int vca_vc_attention_host(const vca_bf16* Q, const vca_bf16* K, const
 
   const size_t row = (size_t)N * d;   // elements per unit
   char* base = (char*)dev_buf;
-  const int nchunks = chunk_count(units, u);
+  const std::vector<int> starts = chunk_starts(units, u);
+  const int nchunks = (int)starts.size() - 1;
   // each call starts with clean status words in both slots' workspaces
   for (int s = 0; s < 2 && !rc; ++s) rc = vca_reset_status(base + (size_t)s * L.total + L.ws, st.comp);
   for (int c = 0; c < nchunks && !rc; ++c) {
     const int s = c & 1;
-    const int u0 = chunk_start(c, units, u), uc = chunk_start(c + 1, units, u) - u0;
+    const int u0 = starts[c], uc = starts[c + 1] - u0;
     char* b = base + (size_t)s * L.total;
     const size_t bytes = (size_t)uc * row * 2;
     // slot s is free once chunk c-2's output has left the device

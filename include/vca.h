@@ -237,10 +237,12 @@ int vca_attention_fwd_skip(const uint8_t* Qq, const float* q_scale, const uint8_
  * vca_attention_fwd), with the copies overlapped with the kernels.  The pages
  * have no counterpart: it serves callers whose activations live in host memory.
  * (b, h) units are independent, so the layer runs in chunks of
- * `heads_per_chunk` units (0 = about eight chunks) through a three-stage
+ * up to `heads_per_chunk` units (0 = a fifth of the layer) through a three-stage
  * pipeline on library-owned streams over two device slots: copy chunk c+1 in,
- * compute chunk c, copy chunk c-1 out.  Results equal the three calls on the
- * whole layer bit for bit.
+ * compute chunk c, copy chunk c-1 out.  Chunk sizes double from one unit up to
+ * heads_per_chunk and the last chunk is one unit, so the transfers nothing
+ * overlaps stay small.  Results equal the three calls on the whole layer bit
+ * for bit.
  *   Q, K, V   [B][H][N][d] bf16, HOST memory (in); page-locked memory
  *             (cudaHostAlloc / cudaHostRegister) is needed for the copies to
  *             overlap -- pageable memory works but serialises them
