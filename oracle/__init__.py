@@ -32,6 +32,9 @@ PLANT_TRUNC = 64
 PLANT_NO_MEAN = 128
 PLANT_BETA0 = 256
 PLANT_NO_RESCALE = 512
+PLANT_NIBBLE = 1024
+PLANT_P_GROUP32 = 2048
+P_GSCALE = 0.125   # NVFP4 tensor scale of the 4-bit variant's probabilities
 BLOCK = 128
 
 _lib = None
@@ -75,6 +78,15 @@ def _declare(L):
     L.vo_attention_head_sage.argtypes = [vp] * 6 + [i32, i32, f64, vp, i32, i32, vp, vp]
     L.vo_attention_head_skip.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, f64, vp, vp, vp]
     L.vo_attention_head_bf16_skip.argtypes = [vp] * 4 + [i32, i32, f64, vp, i32, i32, f64, vp]
+    L.vo_e2m1_decode.restype = f64
+    L.vo_e2m1_decode.argtypes = [ctypes.c_uint8]
+    L.vo_e2m1_encode.restype = ctypes.c_uint8
+    L.vo_e2m1_encode.argtypes = [ctypes.c_float]
+    L.vo_nvfp4_quantize.argtypes = [vp, i64, ctypes.c_float, vp, vp]
+    L.vo_smooth_quantize_head_fp4.argtypes = [vp] * 4 + [i32, i32] + [vp] * 8
+    L.vo_attention_head_fp4.argtypes = [vp] * 6 + [ctypes.c_float, vp, i32, i32, f64, vp, i32, i32, vp, vp]
+    L.vo_p_nvfp4.argtypes = [vp, i32, i32, vp]
+    L.vo_attention_head_fp4_bf16.argtypes = [vp] * 4 + [i32, i32, f64, vp, i32, i32, vp]
     L.vo_exact_attention_head.argtypes = [vp] * 3 + [i32, i32, f64, vp, i32, vp]
     L.vo_num_threads.restype = i32
 
@@ -97,6 +109,26 @@ def e4m3_encode(x) -> np.ndarray:
     out = np.empty(x.shape, dtype=np.uint8)
     lib().vo_e4m3_encode_array(_p(x), _p(out), x.size)
     return out
+
+
+# ------------------------------------------------------------------ E2M1 / NVFP4
+def e2m1_decode_table() -> np.ndarray:
+    return np.array([lib().vo_e2m1_decode(c) for c in range(16)], np.float64)
+
+
+def e2m1_encode(x) -> np.ndarray:
+    x = np.asarray(x, dtype=np.float32)
+    return np.array([lib().vo_e2m1_encode(float(v)) for v in x.ravel()], np.uint8).reshape(x.shape)
+
+
+def nvfp4_quantize(x, G: float):
+    """NVFP4 codes (one nibble per byte) and E4M3 group scales of x[n] in
+    groups of 16 consecutive elements, tensor scale G."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32).ravel())
+    codes = np.empty(x.size, np.uint8)
+    scales = np.empty((x.size + 15) // 16, np.uint8)
+    lib().vo_nvfp4_quantize(_p(x), x.size, float(G), _p(codes), _p(scales))
+    return codes, scales
 
 
 # ------------------------------------------------------------------ ExpCast
@@ -177,6 +209,27 @@ def smooth_quantize_head(Q, K, V, perm):
     return out
 
 
+def smooth_quantize_head_fp4(Q, K, V, perm):
+    """One head of the 4-bit V-Smooth variant: Q/K and block means as the 8-bit
+    prep, the V residual in NVFP4 (VrT4 [d, Np/2] packed, v_sc [d, Np/16],
+    v_gscale)."""
+    Q, K, V = (np.ascontiguousarray(a, dtype=np.uint16) for a in (Q, K, V))
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    N, d = Q.shape
+    nb = (N + BLOCK - 1) // BLOCK
+    Np = nb * BLOCK
+    out = dict(
+        Qq=np.zeros((Np, d), np.uint8), q_scale=np.empty(nb, np.float32),
+        Kq=np.zeros((Np, d), np.uint8), k_scale=np.empty(nb, np.float32),
+        VrT4=np.zeros((d, Np // 2), np.uint8), v_sc=np.zeros((d, Np // 16), np.uint8),
+        v_gscale=np.empty(1, np.float32), v_mean=np.empty((nb, d), np.uint16))
+    lib().vo_smooth_quantize_head_fp4(
+        _p(Q), _p(K), _p(V), _p(perm), N, d, _p(out["Qq"]), _p(out["q_scale"]),
+        _p(out["Kq"]), _p(out["k_scale"]), _p(out["VrT4"]), _p(out["v_sc"]),
+        _p(out["v_gscale"]), _p(out["v_mean"]))
+    return out
+
+
 def sage_quantize_head(Q, K, V):
     """One head of the SAGE-style comparison quantisation (per-token Q,
     per-16-token K after K-mean smoothing, per-channel V; no reordering)."""
@@ -243,6 +296,41 @@ def attention_head_sage(ops: dict, N: int, softmax_scale: float, rows=None, flag
         _p(c["Qq"]), _p(c["q_scale"]), _p(c["Kq"]), _p(c["k_scale"]), _p(c["VcT"]), _p(c["v_chscale"]),
         N, d, float(softmax_scale), _p(rows), rows.shape[0], int(flags), _p(O), _p(lse))
     return O, lse
+
+
+def attention_head_fp4(ops: dict, N: int, softmax_scale: float, rows=None, flags: int = 0):
+    """Attention of the 4-bit variant (dict from ``smooth_quantize_head_fp4``).
+    Returns (O [nrows, d] fp64, lse [nrows])."""
+    rows = _rows(rows, N)
+    d = ops["Qq"].shape[1]
+    O = np.empty((rows.shape[0], d), np.float64)
+    lse = np.empty(rows.shape[0], np.float64)
+    c = {k: np.ascontiguousarray(v) for k, v in ops.items()}
+    lib().vo_attention_head_fp4(
+        _p(c["Qq"]), _p(c["q_scale"]), _p(c["Kq"]), _p(c["k_scale"]), _p(c["VrT4"]), _p(c["v_sc"]),
+        float(c["v_gscale"].ravel()[0]), _p(c["v_mean"]), N, d, float(softmax_scale), _p(rows),
+        rows.shape[0], int(flags), _p(O), _p(lse))
+    return O, lse
+
+
+def p_nvfp4(p, flags: int = 0) -> np.ndarray:
+    """The 4-bit variant's probability quantisation of one key block (n <= 128)."""
+    p = np.ascontiguousarray(np.asarray(p, np.float64).ravel())
+    assert p.size <= BLOCK
+    out = np.empty_like(p)
+    lib().vo_p_nvfp4(_p(p), p.size, int(flags), _p(out))
+    return out
+
+
+def attention_head_fp4_bf16(Q, K, V, perm, softmax_scale: float, rows=None, flags: int = 0):
+    Q, K, V = (np.ascontiguousarray(a, dtype=np.uint16) for a in (Q, K, V))
+    perm = np.ascontiguousarray(perm, dtype=np.int32)
+    N, d = Q.shape
+    rows = _rows(rows, N)
+    O = np.empty((rows.shape[0], d), np.float64)
+    lib().vo_attention_head_fp4_bf16(_p(Q), _p(K), _p(V), _p(perm), N, d, float(softmax_scale),
+                                     _p(rows), rows.shape[0], int(flags), _p(O))
+    return O
 
 
 def exact_attention_head(Q, K, V, softmax_scale: float, rows=None):

@@ -142,6 +142,63 @@ void vo_expcast_array(const float* z, uint8_t* out, int64_t n, int flags) {
     for (int64_t i = 0; i < n; ++i) out[i] = vo_expcast(z[i], flags);
 }
 
+/* ------------------------------------------------------------- E2M1, NVFP4 */
+
+/* E2M1, the element type of NVFP4 ("Accelerating Video Generation with GEMM
+ * Quantization, Attention Quantization and Skip Softmax Attention in
+ * TensorRT-LLM", table of quantisation formats): a sign bit, 2 exponent bits
+ * with bias 1 and 1 mantissa bit; exponent field 0 holds 0 and the subnormal
+ * 0.5; no infinities, no NaN; largest magnitude 6.  Bits 0..2 of a code hold
+ * the magnitude, bit 3 the sign. */
+double vo_e2m1_decode(uint8_t code) {
+    int e = (code >> 1) & 3, m = code & 1;
+    double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return (code & 8) ? -mag : mag;
+}
+
+/* Nearest E2M1 value, ties to the even code, finite values saturating at +-6;
+ * the sign is kept (a negative that rounds to 0 gives 0x8). */
+uint8_t vo_e2m1_encode(float x) {
+    uint8_t sign = signbit(x) ? 8 : 0;
+    double a = fabs((double)x);
+    uint8_t k = 0;
+    for (; k < 7; ++k) {
+        double mid = 0.5 * (vo_e2m1_decode(k) + vo_e2m1_decode((uint8_t)(k + 1)));
+        if (a < mid || (a == mid && (k & 1) == 0)) break;
+    }
+    return sign | k;
+}
+
+/* NVFP4 (same table): E2M1 elements, one E4M3 scale per 16 consecutive
+ * elements, one fp32 scale per tensor.  READING (the pages give the format,
+ * not the rounding recipe): with the tensor scale G (fp32, > 0) a group's
+ * scale is chosen so that its largest element lands on 6, and both quotients
+ * are taken in fp32 as a kernel takes them:
+ *   t = amax_g / (6 G);  sc = e4m3(t);  s = decode(sc)
+ *   code_i = e2m1(x_i * (1 / (s G)))
+ * (one rounding per fp32 product, quotient and reciprocal).  A group whose
+ * scale decodes to 0 gets zero codes.  An element stands for G * s * e2m1(code).
+ * Writes n codes (16 for a whole group), one nibble per byte; returns sc. */
+static uint8_t nvfp4_group(const float* x, int n, float G, uint8_t* codes) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i)
+        if (fabsf(x[i]) > amax) amax = fabsf(x[i]);
+    float t = amax / (6.0f * G);
+    uint8_t sc = vo_e4m3_encode(t);
+    float sg = (float)vo_e4m3_decode(sc) * G;
+    float inv = sg > 0.0f ? 1.0f / sg : 0.0f;
+    for (int i = 0; i < n; ++i) codes[i] = sg > 0.0f ? vo_e2m1_encode(x[i] * inv) : 0;
+    return sc;
+}
+
+void vo_nvfp4_quantize(const float* x, int64_t n, float G, uint8_t* codes, uint8_t* scales) {
+    e4m3_table_init();
+    for (int64_t g = 0; g * 16 < n; ++g) {
+        int len = n - g * 16 < 16 ? (int)(n - g * 16) : 16;
+        scales[g] = nvfp4_group(x + g * 16, len, G, codes + g * 16);
+    }
+}
+
 /* --------------------------------------------------------------- k-means */
 
 /* Squared L2 distance in fp32, channel order 0..d-1, one fmaf per channel.
@@ -266,6 +323,28 @@ static void quant_rows_block(const float* x /* [nv][d] */, int nv, int d,
     for (int i = 0; i < nv * d; ++i) out[i] = vo_e4m3_encode(x[i] * inv);
 }
 
+/* The V block mean of V-Smooth: per channel, the exact fixed-point sum of the
+ * block's nv values, one fp64 division, one rounding to bf16 (mean_out[d]);
+ * xv [nv][d] is replaced in place by the fp32 residual v - mean.  Returns the
+ * residual's largest magnitude. */
+static float v_block_residual(float* xv, int nv, int d, uint16_t* mean_out) {
+    float amax = 0.0f;
+    for (int c = 0; c < d; ++c) {
+        int64_t S = 0;
+        for (int t = 0; t < nv; ++t) S += llrint((double)xv[t * d + c] * 16777216.0);
+        double mean = (double)S / ((double)nv * 16777216.0);
+        uint16_t mb = vo_double_to_bf16_rne(mean);
+        mean_out[c] = mb;
+        float mf = vo_bf16_to_float(mb);
+        for (int t = 0; t < nv; ++t) {
+            float r = xv[t * d + c] - mf;
+            xv[t * d + c] = r;
+            if (fabsf(r) > amax) amax = fabsf(r);
+        }
+    }
+    return amax;
+}
+
 /* V-Smooth on one head ([VCA-news] V-Smooth bullet; [VCA-ru] "Решение";
  * [VCA-mtp] 0.125 bit per value element for the mean):
  *   K and V rows are gathered by the permutation; in each block of 128
@@ -298,21 +377,7 @@ void vo_smooth_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_
         }
         quant_rows_block(xq, nv, d, Qq + (int64_t)n0 * d, &q_scale[b]);
         quant_rows_block(xk, nv, d, Kq + (int64_t)n0 * d, &k_scale[b]);
-        /* V block mean, stored as bf16 */
-        float amax = 0.0f;
-        for (int c = 0; c < d; ++c) {
-            int64_t S = 0;
-            for (int t = 0; t < nv; ++t) S += llrint((double)xv[t * d + c] * 16777216.0);
-            double mean = (double)S / ((double)nv * 16777216.0);
-            uint16_t mb = vo_double_to_bf16_rne(mean);
-            v_mean[(int64_t)b * d + c] = mb;
-            float mf = vo_bf16_to_float(mb);
-            for (int t = 0; t < nv; ++t) {
-                float r = xv[t * d + c] - mf;
-                xv[t * d + c] = r;
-                if (fabsf(r) > amax) amax = fabsf(r);
-            }
-        }
+        float amax = v_block_residual(xv, nv, d, v_mean + (int64_t)b * d);
         int e = vo_v_exponent(amax);
         v_exp[b] = (int8_t)e;
         for (int c = 0; c < d; ++c)
@@ -320,6 +385,70 @@ void vo_smooth_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_
                 VrT[(int64_t)c * Np + n0 + t] = vo_e4m3_encode(ldexpf(xv[t * d + c], -e));
         free(xq); free(xk); free(xv);
     }
+}
+
+/* The 4-bit V-Smooth variant ([VCA-mtp] abstract and Chinese section: a 4-bit
+ * V-Smooth runs on workstation cards; ExpCast is 8-bit only because NVFP4 has
+ * no single affine log-to-code map).  READING: the 4-bit change is confined to
+ * the PV product -- Q and K are quantised exactly as in the 8-bit variant, the
+ * V block means are the same bf16 means, and only the residual r = v - mean
+ * moves from E4M3 to NVFP4, in groups of 16 consecutive permuted tokens of one
+ * channel (the key dimension is the PV contraction dimension), with one tensor
+ * scale per head: G = amax_head(|r|) / (6 * 448), G = 1 for an all-zero
+ * residual.  Outputs besides the 8-bit ones:
+ *   VrT4 [d][Np/2]: token j of channel c in byte c*Np/2 + j/2, low nibble for
+ *                   even j; v_sc [d][Np/16]: E4M3 group scales; *v_gscale = G.
+ * Padding tokens (j >= N) have zero codes; groups wholly past N zero scales. */
+void vo_smooth_quantize_head_fp4(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                 const int32_t* perm, int N, int d,
+                                 uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                                 uint8_t* VrT4, uint8_t* v_sc, float* v_gscale, uint16_t* v_mean) {
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    int64_t Np = (int64_t)nb * VO_BLOCK;
+    float* R = (float*)malloc((size_t)N * d * sizeof(float));   /* residuals, permuted order */
+    float* bmax = (float*)malloc((size_t)nb * sizeof(float));
+#pragma omp parallel for schedule(dynamic)
+    for (int b = 0; b < nb; ++b) {
+        int n0 = b * VO_BLOCK;
+        int nv = N - n0 < VO_BLOCK ? N - n0 : VO_BLOCK;
+        float* xq = (float*)malloc((size_t)VO_BLOCK * d * sizeof(float));
+        float* xk = (float*)malloc((size_t)VO_BLOCK * d * sizeof(float));
+        for (int t = 0; t < nv; ++t) {
+            int64_t src = perm[n0 + t];
+            for (int c = 0; c < d; ++c) {
+                xq[t * d + c] = vo_bf16_to_float(Q[(int64_t)(n0 + t) * d + c]);
+                xk[t * d + c] = vo_bf16_to_float(K[src * d + c]);
+                R[(int64_t)(n0 + t) * d + c] = vo_bf16_to_float(V[src * d + c]);
+            }
+        }
+        quant_rows_block(xq, nv, d, Qq + (int64_t)n0 * d, &q_scale[b]);
+        quant_rows_block(xk, nv, d, Kq + (int64_t)n0 * d, &k_scale[b]);
+        bmax[b] = v_block_residual(R + (int64_t)n0 * d, nv, d, v_mean + (int64_t)b * d);
+        free(xq); free(xk);
+    }
+    float amax = 0.0f;
+    for (int b = 0; b < nb; ++b)
+        if (bmax[b] > amax) amax = bmax[b];
+    float G = amax > 0.0f ? amax / 2688.0f : 1.0f;
+    *v_gscale = G;
+    memset(VrT4, 0, (size_t)d * (Np / 2));
+    memset(v_sc, 0, (size_t)d * (Np / 16));
+#pragma omp parallel for schedule(static)
+    for (int c = 0; c < d; ++c) {
+        float x[16];
+        uint8_t codes[16];
+        for (int j0 = 0; j0 < N; j0 += 16) {
+            int n = N - j0 < 16 ? N - j0 : 16;
+            for (int i = 0; i < n; ++i) x[i] = R[(int64_t)(j0 + i) * d + c];
+            v_sc[(int64_t)c * (Np / 16) + j0 / 16] = nvfp4_group(x, n, G, codes);
+            for (int i = 0; i < n; ++i) {
+                int64_t j = j0 + i;
+                VrT4[(int64_t)c * (Np / 2) + j / 2] |= (uint8_t)(codes[i] << (4 * (j & 1)));
+            }
+        }
+    }
+    free(R);
+    free(bmax);
 }
 
 /* SAGE-style quantisation, the comparison recipe of "Accelerating Video
@@ -424,6 +553,34 @@ void vo_sage_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_t*
  * READING: the pages name online softmax but not its rescale rule; this one
  * (a reference that lags the running maximum by at most VO_LAG octaves) keeps
  * every code <= 56 + 8*(VO_HEADROOM + VO_LAG) = 120 < 126. */
+/* Internal flag: the 4-bit variant's probabilities (see p_nvfp4_block). */
+#define VO_P_NVFP4 (1 << 16)
+
+/* READING: the probabilities of the 4-bit variant are bounded by
+ * 2^(VO_HEADROOM + VO_LAG) = 256 by the reference rule, so their NVFP4 tensor
+ * scale is the fixed power of two 2^-3 (the bound lands on a group scale of
+ * 341 <= 448 with no pass over the data, and a power of two cancels exactly
+ * against the row sum). */
+#define VO_P_GSCALE 0.125f
+
+/* NVFP4 quantisation of one key block of a row's probabilities, in place
+ * (the 4-bit variant; ExpCast does not apply to 4 bits, so p is computed as
+ * an exponential, rounded once to fp32, then quantised in groups of 16 keys
+ * with tensor scale VO_P_GSCALE; the row sum then adds the dequantised values,
+ * as the PV product does). */
+static void p_nvfp4_block(double* pb, int n, int flags) {
+    int gsz = (flags & VO_PLANT_P_GROUP32) ? 32 : 16;
+    float x[32];
+    uint8_t codes[32];
+    for (int g0 = 0; g0 < n; g0 += gsz) {
+        int len = n - g0 < gsz ? n - g0 : gsz;
+        for (int i = 0; i < len; ++i) x[i] = (float)pb[g0 + i];
+        uint8_t sc = nvfp4_group(x, len, VO_P_GSCALE, codes);
+        double sg = vo_e4m3_decode(sc) * (double)VO_P_GSCALE;
+        for (int i = 0; i < len; ++i) pb[g0 + i] = sg * vo_e2m1_decode(codes[i]);
+    }
+}
+
 static void attn_row(const double* q, double qs, const double* kh, const double* ks,
                      const double* rh, const int* vexp, const double* mu, int N, int d,
                      double softmax_scale, int flags, double skip_log2, double* O, double* lse,
@@ -465,11 +622,11 @@ static void attn_row(const double* q, double qs, const double* kh, const double*
             n = nblk;
         }
         double lb = 0.0;
-        double pv[512];
+        double pv[512], pb[VO_BLOCK];
         for (int c = 0; c < d; ++c) pv[c] = 0.0;
         for (int j = j0; j < j1; ++j) {
             double p;
-            if (flags & VO_EXACT_EXP) {
+            if (flags & (VO_EXACT_EXP | VO_P_NVFP4)) {
                 p = exp2(z[j] - (n + VO_PHI) + VO_HEADROOM);
             } else {
                 /* = 8(z - m) + 55.65 + 8*VO_HEADROOM with m = n + phi */
@@ -480,6 +637,11 @@ static void attn_row(const double* q, double qs, const double* kh, const double*
                 if (r > 126.0) r = 126.0;
                 p = vo_e4m3_decode((uint8_t)r);
             }
+            pb[j - j0] = p;
+        }
+        if ((flags & VO_P_NVFP4) && !(flags & VO_IDENTITY_QUANT)) p_nvfp4_block(pb, j1 - j0, flags);
+        for (int j = j0; j < j1; ++j) {
+            double p = pb[j - j0];
             lb += p;
             for (int c = 0; c < d; ++c) pv[c] += p * rh[(int64_t)j * d + c];
         }
@@ -589,6 +751,76 @@ void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8
     for (int r = 0; r < nrows; ++r)
         for (int c = 0; c < d; ++c) O[(int64_t)r * d + c] *= v_chscale[c];
     free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
+}
+
+/* The 4-bit variant's probability step on its own: n <= 128 consecutive keys
+ * of one row (a key block), p[] the fp64 probabilities relative to the
+ * reference; out[] the dequantised NVFP4 values the row sum and PV use. */
+void vo_p_nvfp4(const double* p, int n, int flags, double* out) {
+    for (int i = 0; i < n; ++i) out[i] = p[i];
+    p_nvfp4_block(out, n, flags);
+}
+
+/* Attention of the 4-bit variant: the 8-bit row algorithm (online reference,
+ * mean restore from the row sums) with NVFP4 probabilities (p_nvfp4_block)
+ * and the NVFP4 V residual of vo_smooth_quantize_head_fp4, dequantised as
+ * G * s * e2m1(code). */
+void vo_attention_head_fp4(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                           const float* k_scale, const uint8_t* VrT4, const uint8_t* v_sc,
+                           float v_gscale, const uint16_t* v_mean, int N, int d, double softmax_scale,
+                           const int32_t* rows, int nrows, int flags, double* O, double* lse) {
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    int64_t Np = (int64_t)nb * VO_BLOCK;
+    double* qh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* kh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* rh = (double*)malloc((size_t)N * d * sizeof(double));
+    double* qs = (double*)malloc((size_t)N * sizeof(double));
+    double* ks = (double*)malloc((size_t)N * sizeof(double));
+    double* mu = (double*)malloc((size_t)nb * d * sizeof(double));
+    int* ve = (int*)calloc((size_t)nb, sizeof(int));
+    for (int j = 0; j < N; ++j) {
+        qs[j] = q_scale[j / VO_BLOCK];
+        ks[j] = k_scale[j / VO_BLOCK];
+        for (int c = 0; c < d; ++c) {
+            qh[(int64_t)j * d + c] = vo_e4m3_decode(Qq[(int64_t)j * d + c]);
+            kh[(int64_t)j * d + c] = vo_e4m3_decode(Kq[(int64_t)j * d + c]);
+            uint8_t byte = VrT4[(int64_t)c * (Np / 2) + j / 2];
+            int hi = (j & 1) ^ ((flags & VO_PLANT_NIBBLE) ? 1 : 0);
+            uint8_t code = hi ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+            double s = vo_e4m3_decode(v_sc[(int64_t)c * (Np / 16) + j / 16]);
+            rh[(int64_t)j * d + c] = (double)v_gscale * s * vo_e2m1_decode(code);
+        }
+    }
+    for (int b = 0; b < nb; ++b)
+        for (int c = 0; c < d; ++c) mu[(int64_t)b * d + c] = vo_bf16_to_float(v_mean[(int64_t)b * d + c]);
+    attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags | VO_P_NVFP4, -INFINITY, O,
+              lse, NULL);
+    free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
+}
+
+/* The 4-bit variant straight from bf16 Q/K/V and a permutation; with
+ * VO_IDENTITY_QUANT no quantiser rounds (operands exact, exact fp64 block means,
+ * exact probabilities), which must give exact softmax attention. */
+void vo_attention_head_fp4_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                const int32_t* perm, int N, int d, double softmax_scale,
+                                const int32_t* rows, int nrows, int flags, double* O) {
+    if (flags & VO_IDENTITY_QUANT) {
+        vo_attention_head_bf16_skip(Q, K, V, perm, N, d, softmax_scale, rows, nrows, flags | VO_P_NVFP4, 0.0, O);
+        return;
+    }
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    int64_t Np = (int64_t)nb * VO_BLOCK;
+    uint8_t* Qq = (uint8_t*)malloc((size_t)Np * d);
+    uint8_t* Kq = (uint8_t*)malloc((size_t)Np * d);
+    uint8_t* VrT4 = (uint8_t*)malloc((size_t)d * (Np / 2));
+    uint8_t* vsc = (uint8_t*)malloc((size_t)d * (Np / 16));
+    float* qsc = (float*)malloc((size_t)nb * sizeof(float));
+    float* ksc = (float*)malloc((size_t)nb * sizeof(float));
+    uint16_t* vm = (uint16_t*)malloc((size_t)nb * d * sizeof(uint16_t));
+    float G = 1.0f;
+    vo_smooth_quantize_head_fp4(Q, K, V, perm, N, d, Qq, qsc, Kq, ksc, VrT4, vsc, &G, vm);
+    vo_attention_head_fp4(Qq, qsc, Kq, ksc, VrT4, vsc, G, vm, N, d, softmax_scale, rows, nrows, flags, O, NULL);
+    free(Qq); free(Kq); free(VrT4); free(vsc); free(qsc); free(ksc); free(vm);
 }
 
 void vo_attention_head_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t* V,

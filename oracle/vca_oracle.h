@@ -39,6 +39,8 @@ extern "C" {
 #define VO_PLANT_NO_MEAN   128 /* planted mistake: drop the rowsum*mean restore term */
 #define VO_PLANT_BETA0     256 /* planted mistake: addend 56 instead of 56 + beta    */
 #define VO_PLANT_NO_RESCALE 512 /* planted mistake: reference moves without rescaling */
+#define VO_PLANT_NIBBLE    1024 /* planted mistake (4-bit): V nibbles read high first  */
+#define VO_PLANT_P_GROUP32 2048 /* planted mistake (4-bit): P groups of 32 keys       */
 
 /* E4M3 (OCP FP8: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
  * no infinities, NaN = S.1111.111, largest finite 448). */
@@ -49,6 +51,14 @@ void    vo_e4m3_encode_array(const float* x, uint8_t* out, int64_t n);
 /* ExpCast-FP8 on a log2-domain, max-subtracted score z. */
 uint8_t vo_expcast(float z, int flags);
 void    vo_expcast_array(const float* z, uint8_t* out, int64_t n, int flags);
+
+/* E2M1 (NVFP4 element: sign, 2 exponent bits with bias 1, 1 mantissa bit;
+ * magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6), nearest with ties to even, saturating. */
+double  vo_e2m1_decode(uint8_t code);
+uint8_t vo_e2m1_encode(float x);
+/* NVFP4 quantisation of x[n] in groups of 16 with tensor scale G: codes[n] (one
+ * nibble per byte) and scales[ceil(n/16)] E4M3 codes. */
+void    vo_nvfp4_quantize(const float* x, int64_t n, float G, uint8_t* codes, uint8_t* scales);
 
 /* bf16 helpers. */
 float    vo_bf16_to_float(uint16_t b);
@@ -107,6 +117,27 @@ void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8
                             const float* k_scale, const uint8_t* VcT, const float* v_chscale,
                             int N, int d, double softmax_scale, const int32_t* rows, int nrows,
                             int flags, double* O, double* lse);
+
+/* The 4-bit V-Smooth variant ("Nunchux AI Introduces VC-Attention...",
+ * abstract: 4-bit V-Smooth on workstation cards; ExpCast is 8-bit only).
+ * Q, K, v_mean as in vo_smooth_quantize_head; the V residual in NVFP4:
+ * VrT4 [d][Np/2] (low nibble = even token), v_sc [d][Np/16] E4M3 group
+ * scales, *v_gscale the head's fp32 tensor scale. */
+void vo_smooth_quantize_head_fp4(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                 const int32_t* perm, int N, int d,
+                                 uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                                 uint8_t* VrT4, uint8_t* v_sc, float* v_gscale, uint16_t* v_mean);
+/* Attention on those operands with NVFP4 probabilities (16-key groups, tensor
+ * scale 2^-3); O [nrows][d] fp64, lse [nrows] nullable. */
+void vo_attention_head_fp4(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                           const float* k_scale, const uint8_t* VrT4, const uint8_t* v_sc,
+                           float v_gscale, const uint16_t* v_mean, int N, int d, double softmax_scale,
+                           const int32_t* rows, int nrows, int flags, double* O, double* lse);
+/* Its probability step alone: n <= 128 keys of one row, out = dequantised. */
+void vo_p_nvfp4(const double* p, int n, int flags, double* out);
+void vo_attention_head_fp4_bf16(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                const int32_t* perm, int N, int d, double softmax_scale,
+                                const int32_t* rows, int nrows, int flags, double* O);
 
 /* Same algorithm, straight from bf16 Q/K/V and a permutation; with
  * VO_IDENTITY_QUANT the quantisers are the identity (for reductions). */
