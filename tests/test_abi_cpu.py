@@ -65,3 +65,57 @@ def test_product_path_does_not_import_the_oracle():
                 txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in txt and "from oracle" not in txt, f
                 assert "vca_oracle" not in txt and "liboracle" not in txt, f
+
+
+FAKE = ctypes.c_void_p(0x10000)       # a 16-byte-aligned address that is never dereferenced
+FAKE_ODD = ctypes.c_void_p(0x10001)
+
+
+def test_attention_variants_validate_on_the_host(L):
+    ops = [FAKE] * 7
+    # skip_lambda must lie in [0, 1)
+    rc = L.vca_attention_fwd_skip(*ops, 1, 1, 300, 128, 0.1, 1.0, FAKE, None, None, FAKE, 256, None)
+    assert rc == vca.ERR_INVALID and b"skip_lambda" in L.vca_last_error()
+    rc = L.vca_attention_fwd_skip(*ops, 1, 1, 300, 128, 0.1, -0.5, FAKE, None, None, FAKE, 256, None)
+    assert rc == vca.ERR_INVALID
+    # alignment of the TMA-fed tensors, softmax scale, grid limit, workspace
+    rc = L.vca_attention_fwd(FAKE_ODD, *ops[1:], 1, 1, 300, 128, 0.1, FAKE, None, FAKE, 256, None)
+    assert rc == vca.ERR_INVALID and b"aligned" in L.vca_last_error()
+    rc = L.vca_attention_fwd(*ops, 1, 1, 300, 128, 0.0, FAKE, None, FAKE, 256, None)
+    assert rc == vca.ERR_INVALID and b"softmax_scale" in L.vca_last_error()
+    rc = L.vca_attention_fwd(*ops, 256, 256, 300, 128, 0.1, FAKE, None, FAKE, 256, None)
+    assert rc == vca.ERR_INVALID
+    rc = L.vca_attention_fwd(*ops, 1, 1, 300, 128, 0.1, FAKE, None, FAKE, 16, None)
+    assert rc == vca.ERR_WORKSPACE
+    # SAGE operands: the per-channel V scale is required; d must be 128
+    rc = L.vca_attention_fwd_sage(*[FAKE] * 5, None, 1, 1, 300, 128, 0.1, FAKE, None, FAKE, 256, None)
+    assert rc == vca.ERR_INVALID
+    rc = L.vca_attention_fwd_sage(*[FAKE] * 6, 1, 1, 300, 64, 0.1, FAKE, None, FAKE, 256, None)
+    assert rc == vca.ERR_UNSUPPORTED
+    rc = L.vca_sage_quantize_qkv(FAKE, FAKE, FAKE, 1, 1, 300, 96, *[FAKE] * 7, FAKE, 1 << 20, None)
+    assert rc == vca.ERR_UNSUPPORTED
+
+
+def test_host_pipeline_validates_and_sizes_on_the_host(L):
+    B, H, N, k = 1, 8, 1000, 32
+    full = L.vca_vc_attention_host_buffer_size(B, H, N, 128, k, 0)
+    one = L.vca_vc_attention_host_buffer_size(B, H, N, 128, k, 1)
+    all8 = L.vca_vc_attention_host_buffer_size(B, H, N, 128, k, 8)
+    # two slots, each sized for one chunk: more heads per chunk, more memory
+    assert 0 < one < full <= all8
+    assert L.vca_vc_attention_host_buffer_size(B, H, N, 128, k, 100) == all8
+    # at least Q, K, V, O in bf16 and the three FP8 operands per slot
+    assert one >= 2 * (4 * N * 128 * 2 + 3 * N * 128)
+    for bad in ((0, H, N, 128, k, 0), (B, H, N, 64, k, 0), (B, H, N, 128, 0, 0), (B, H, N, 128, 1000, 0)):
+        assert L.vca_vc_attention_host_buffer_size(*bad) == 0
+    host = [FAKE] * 3
+    rc = L.vca_vc_attention_host(None, FAKE, FAKE, B, H, N, 128, k, 3, 0.1, FAKE, 0, FAKE, full, None)
+    assert rc == vca.ERR_INVALID
+    rc = L.vca_vc_attention_host(*host, B, H, N, 64, k, 3, 0.1, FAKE, 0, FAKE, full, None)
+    assert rc == vca.ERR_UNSUPPORTED
+    rc = L.vca_vc_attention_host(*host, B, H, N, 128, k, 0, 0.1, FAKE, 0, FAKE, full, None)
+    assert rc == vca.ERR_INVALID
+    rc = L.vca_vc_attention_host(*host, B, H, N, 128, k, 3, 0.1, FAKE, -1, FAKE, full, None)
+    assert rc == vca.ERR_INVALID
+    rc = L.vca_vc_attention_host(*host, B, H, N, 128, k, 3, 0.1, FAKE, 0, FAKE, full - 1, None)
+    assert rc == vca.ERR_WORKSPACE and b"too small" in L.vca_last_error()
