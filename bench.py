@@ -392,11 +392,62 @@ def run_ours(args, world, rank, local):
                         "quantise_ms": round(quant_ms, 3),
                         "grouping_frac_of_attention": round(n_regroup * group_ms / (S * t_attn * 1e3), 4),
                         "prep_frac_of_attention": round((n_regroup * group_ms + S * quant_ms) / (S * t_attn * 1e3), 4)}
+    # share of block energy the V block mean carries (what V-Smooth removes before
+    # quantising), in three token orders; perm is the product path's grouping
+    line["block_mean_energy"] = dict(block_mean_energy(V, perm, w.grid), heads=B * H,
+                                     cube="2x8x8 tokens of the (t, h, w) latent grid")
     pb = prep_algorithmic_bytes(w)
     line["prep_roofline"] = {"bound": "hbm", "algorithmic_bytes": pb,
                              "achieved": round(pb / (prep_ms / 1e3) / 1e9, 1), "unit": "GB/s",
                              "peak": peaks["hbm_gbs"], "frac": round(pb / (prep_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
     return line, (Q, K, V, w)
+
+
+def group_mean_energy(v: torch.Tensor, gid: torch.Tensor, ngroups: int) -> float:
+    """Share of the energy of one head's value tokens v [N, d] that their group
+    means carry, sum_g n_g |mean_g|^2 / sum_j |v_j|^2: what subtracting the
+    means removes, since sum |v|^2 = sum_g n_g |mean_g|^2 + sum |v - mean|^2."""
+    v = v.double()
+    sums = torch.zeros(ngroups, v.shape[1], dtype=torch.float64, device=v.device).index_add_(0, gid, v)
+    cnt = torch.bincount(gid, minlength=ngroups).double()
+    keep = cnt > 0
+    carried = ((sums[keep] ** 2).sum(1) / cnt[keep]).sum()
+    return float(carried / (v * v).sum())
+
+
+def cube_groups(grid, N: int, device, cube=(2, 8, 8)):
+    """Static spatiotemporal cubes of the latent grid (tokens flattened t-major):
+    2 x 8 x 8 = 128 tokens, ragged at the grid's edges.  Returns (gid, ngroups)."""
+    T, Hg, Wg = grid
+    n = torch.arange(N, device=device)
+    t, rem = n // (Hg * Wg), n % (Hg * Wg)
+    h, w = rem // Wg, rem % Wg
+    ct, ch, cw = cube
+    nh, nw = -(-Hg // ch), -(-Wg // cw)
+    gid = ((t // ct) * nh + h // ch) * nw + w // cw
+    return gid, -(-T // ct) * nh * nw
+
+
+def block_mean_energy(V: torch.Tensor, perm: torch.Tensor, grid, block: int = 128) -> dict:
+    """Energy share of the 128-token block means of V, averaged over heads, with
+    the tokens in sequence order, in static cubes of the latent grid, and in
+    the k-means order of perm ("Nunchux AI Introduces VC-Attention ...",
+    abstract: 8 % / 12 % / 36 % over 100 Wan2.2 heads)."""
+    N = V.shape[-2]
+    Vh = V.reshape(-1, N, V.shape[-1])
+    P = perm.reshape(-1, N)
+    nb = -(-N // block)
+    seq = torch.arange(N, device=V.device) // block
+    cube = cube_groups(grid, N, V.device) if grid else None
+    out = {"sequence": [], "static_cube": [], "sorted": []}
+    for h in range(Vh.shape[0]):
+        out["sequence"].append(group_mean_energy(Vh[h], seq, nb))
+        if cube is not None:
+            out["static_cube"].append(group_mean_energy(Vh[h], *cube))
+        srt = torch.empty(N, dtype=torch.long, device=V.device)
+        srt[P[h].long()] = seq          # token perm[i] sits at sorted position i
+        out["sorted"].append(group_mean_energy(Vh[h], srt, nb))
+    return {k: round(statistics.mean(x), 4) for k, x in out.items() if x}
 
 
 def fp8_gemm_ceiling(dev, n=8192, reps=10):
