@@ -102,6 +102,21 @@ std::vector<int> chunk_starts(int units, int u) {
   return starts;
 }
 
+// The seven events of one call (start, and per slot: input landed, compute
+// done, output copied), destroyed on every return path.
+struct Events {
+  cudaEvent_t e[7] = {};
+  bool create() {
+    for (cudaEvent_t& x : e)
+      if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) return false;
+    return true;
+  }
+  ~Events() {
+    for (cudaEvent_t x : e)
+      if (x) cudaEventDestroy(x);
+  }
+};
+
 int units_per_chunk(int units, int heads_per_chunk) {
   if (heads_per_chunk > 0) return heads_per_chunk < units ? heads_per_chunk : units;
   const int u = (units + 4) / 5;   // about five chunks at full size, after the doubling ramp
@@ -134,14 +149,9 @@ extern "C" int vca_vc_attention_host(const vca_bf16* Q, const vca_bf16* K, const
   if (rc) return rc;
 
   // the pipeline starts after the work already queued on the caller's stream
-  cudaEvent_t start, ev_in[2], ev_done[2], ev_free[2];
-  if (cudaEventCreateWithFlags(&start, cudaEventDisableTiming) != cudaSuccess)
-    return fail(VCA_ERR_CUDA, "%s: cannot create events", fn);
-  for (int i = 0; i < 2; ++i)
-    if (cudaEventCreateWithFlags(&ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ev_done[i], cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ev_free[i], cudaEventDisableTiming) != cudaSuccess)
-      return fail(VCA_ERR_CUDA, "%s: cannot create events", fn);
+  Events evs;
+  if (!evs.create()) return fail(VCA_ERR_CUDA, "%s: cannot create events", fn);
+  cudaEvent_t start = evs.e[0], *ev_in = evs.e + 1, *ev_done = evs.e + 3, *ev_free = evs.e + 5;
   cudaEventRecord(start, (cudaStream_t)stream);
   cudaStreamWaitEvent(st.h2d, start, 0);
   cudaStreamWaitEvent(st.comp, start, 0);
@@ -195,12 +205,6 @@ extern "C" int vca_vc_attention_host(const vca_bf16* Q, const vca_bf16* K, const
   const bool sync_ok = cudaStreamSynchronize(st.h2d) == cudaSuccess &&
                        cudaStreamSynchronize(st.comp) == cudaSuccess &&
                        cudaStreamSynchronize(st.d2h) == cudaSuccess;
-  cudaEventDestroy(start);
-  for (int i = 0; i < 2; ++i) {
-    cudaEventDestroy(ev_in[i]);
-    cudaEventDestroy(ev_done[i]);
-    cudaEventDestroy(ev_free[i]);
-  }
   if (rc) return rc;
   if (!sync_ok) return fail(VCA_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(cudaGetLastError()));
   // device-side errors of either slot (timeouts, non-finite inputs)
