@@ -35,6 +35,7 @@ EXPORTED = [
     "vca_bf16_attention_workspace_size", "vca_bf16_attention_fwd", "vca_schedule_regroup",
     "vca_attention_fwd_skip", "vca_vc_attention_host_buffer_size", "vca_vc_attention_host",
     "vca_sage_quantize_workspace_size", "vca_sage_quantize_qkv", "vca_attention_fwd_sage",
+    "vca_smooth_quantize_fp4_workspace_size", "vca_smooth_quantize_qkv_fp4",
 ]
 
 
@@ -78,6 +79,9 @@ def lib() -> ctypes.CDLL:
         L.vca_sage_quantize_workspace_size.argtypes = [i32, i32, i32]
         L.vca_sage_quantize_qkv.argtypes = [vp, vp, vp] + [i32] * 4 + [vp] * 7 + [vp, sz, vp]
         L.vca_attention_fwd_sage.argtypes = [vp] * 6 + [i32] * 4 + [f32, vp, vp, vp, sz, vp]
+        L.vca_smooth_quantize_fp4_workspace_size.restype = sz
+        L.vca_smooth_quantize_fp4_workspace_size.argtypes = [i32, i32, i32]
+        L.vca_smooth_quantize_qkv_fp4.argtypes = [vp] * 4 + [i32] * 4 + [vp] * 8 + [vp, sz, vp]
         L.vca_vc_attention_host_buffer_size.restype = sz
         L.vca_vc_attention_host_buffer_size.argtypes = [i32] * 6
         L.vca_vc_attention_host.argtypes = [vp, vp, vp] + [i32] * 6 + [f32, vp, i32, vp, sz, vp]
@@ -214,6 +218,33 @@ def smooth_quantize(Q, K, V, perm, out=None, ws: Workspace | None = None, stream
         _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), B, H, N, d, BLOCK, _ptr(o["Qq"]), _ptr(o["q_scale"]),
         _ptr(o["Kq"]), _ptr(o["k_scale"]), _ptr(o["VrT"]), _ptr(o["v_exp"]), _ptr(o["v_mean"]),
         ws.ptr, ws.nbytes, _stream(stream)))
+    return o
+
+
+def smooth_quantize_fp4(Q, K, V, perm, out=None, ws: Workspace | None = None, stream=None) -> dict:
+    """4-bit V-Smooth prep: Q/K and block means as ``smooth_quantize``, the V
+    residual in NVFP4 (VrT4 [B,H,d,Np/2] packed codes, v_sc [B,H,d,Np/16] E4M3
+    group scales, v_gscale [B,H] fp32 head scales)."""
+    B, H, N, d = _bhnd(Q)
+    assert K.shape == Q.shape and V.shape == Q.shape
+    assert perm.is_cuda and perm.dtype == torch.int32 and perm.shape == (B, H, N) and perm.is_contiguous()
+    nb = (N + BLOCK - 1) // BLOCK
+    Np = nb * BLOCK
+    dev = Q.device
+    u8, f32 = torch.uint8, torch.float32
+    o = out or dict(
+        Qq=torch.empty(B, H, Np, d, dtype=u8, device=dev), q_scale=torch.empty(B, H, nb, dtype=f32, device=dev),
+        Kq=torch.empty(B, H, Np, d, dtype=u8, device=dev), k_scale=torch.empty(B, H, nb, dtype=f32, device=dev),
+        VrT4=torch.empty(B, H, d, Np // 2, dtype=u8, device=dev),
+        v_sc=torch.empty(B, H, d, Np // 16, dtype=u8, device=dev),
+        v_gscale=torch.empty(B, H, dtype=f32, device=dev),
+        v_mean=torch.empty(B, H, nb, d, dtype=torch.bfloat16, device=dev))
+    need = lib().vca_smooth_quantize_fp4_workspace_size(B, H, N)
+    ws = (ws or Workspace(need, dev)).ensure(need)
+    _check(lib().vca_smooth_quantize_qkv_fp4(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(perm), B, H, N, d, _ptr(o["Qq"]), _ptr(o["q_scale"]),
+        _ptr(o["Kq"]), _ptr(o["k_scale"]), _ptr(o["VrT4"]), _ptr(o["v_sc"]), _ptr(o["v_gscale"]),
+        _ptr(o["v_mean"]), ws.ptr, ws.nbytes, _stream(stream)))
     return o
 
 

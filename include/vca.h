@@ -186,6 +186,31 @@ int vca_smooth_quantize_qkv(const vca_bf16* Q, const vca_bf16* K, const vca_bf16
 
 /* ------------------------------------------------------------------ attention */
 
+/* 4-bit V-Smooth quantisation ([VCA-mtp] abstract: the 4-bit V-Smooth of the
+ * workstation parts; NVFP4 per [TRT-blog], table of quantisation formats:
+ * E2M1 elements, one E4M3 scale per 16 elements, one fp32 scale per tensor).
+ * Q, K, q_scale, k_scale and v_mean are exactly those of
+ * vca_smooth_quantize_qkv; only the V residual r = V - v_mean changes, to NVFP4
+ * in groups of 16 consecutive permuted tokens of one channel:
+ *   v_gscale[b][h] = G = max|r| over the head / (6 * 448)  (1 if r == 0)
+ *   group scale    sc = e4m3(max|r_group| / (6 G))
+ *   codes          e2m1(r * (1 / (decode(sc) * G)))   (nearest, ties to the
+ *                  even code, saturating at +-6; sign in bit 3)
+ * every product, quotient and reciprocal rounded once in fp32; a group whose
+ * scale decodes to 0 has zero codes.  Layouts per (b, h):
+ *   VrT4 [d][Np/2] u8: token j of channel c in byte c*Np/2 + j/2, low nibble
+ *        for even j; v_sc [d][Np/16] u8 E4M3 group scales; v_gscale fp32.
+ * Padding tokens have zero codes, groups wholly past N zero scales.  Q, K, V,
+ * Qq, Kq, VrT4 and v_sc 16-byte aligned; the workspace (status word and one
+ * maximum per head) of vca_smooth_quantize_fp4_workspace_size() bytes.  Same
+ * errors as vca_smooth_quantize_qkv. */
+size_t vca_smooth_quantize_fp4_workspace_size(int B, int H, int N);
+int vca_smooth_quantize_qkv_fp4(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V,
+                                const int32_t* perm, int B, int H, int N, int d, uint8_t* Qq,
+                                float* q_scale, uint8_t* Kq, float* k_scale, uint8_t* VrT4,
+                                uint8_t* v_sc, float* v_gscale, vca_bf16* v_mean, void* ws,
+                                size_t ws_bytes, vca_stream_t stream);
+
 size_t vca_attention_workspace_size(int B, int H, int N);
 
 /* ExpCast-FP8 attention forward, non-causal self-attention ([VCA-news]:

@@ -119,3 +119,20 @@ def test_host_pipeline_validates_and_sizes_on_the_host(L):
     assert rc == vca.ERR_INVALID
     rc = L.vca_vc_attention_host(*host, B, H, N, 128, k, 3, 0.1, FAKE, 0, FAKE, full - 1, None)
     assert rc == vca.ERR_WORKSPACE and b"too small" in L.vca_last_error()
+
+
+def test_fp4_prep_validates_on_the_host(L):
+    assert L.vca_smooth_quantize_fp4_workspace_size(1, 40, 75600) == 256 + 256
+    assert L.vca_smooth_quantize_fp4_workspace_size(2, 100, 10) == 256 + 1024
+    assert L.vca_smooth_quantize_fp4_workspace_size(0, 1, 1) == 0
+    outs = [FAKE] * 8
+    rc = L.vca_smooth_quantize_qkv_fp4(FAKE, FAKE, FAKE, FAKE, 1, 1, 300, 64, *outs, FAKE, 1 << 20, None)
+    assert rc == vca.ERR_UNSUPPORTED
+    rc = L.vca_smooth_quantize_qkv_fp4(FAKE, FAKE, FAKE, FAKE, 1, 1, 300, 128, *outs[:6], None, outs[7],
+                                       FAKE, 1 << 20, None)
+    assert rc == vca.ERR_INVALID and b"null" in L.vca_last_error()
+    rc = L.vca_smooth_quantize_qkv_fp4(FAKE, FAKE, FAKE, FAKE, 1, 1, 300, 128, *outs[:5], FAKE_ODD, *outs[6:],
+                                       FAKE, 1 << 20, None)
+    assert rc == vca.ERR_INVALID and b"aligned" in L.vca_last_error()
+    rc = L.vca_smooth_quantize_qkv_fp4(FAKE, FAKE, FAKE, FAKE, 1, 1, 300, 128, *outs, FAKE, 300, None)
+    assert rc == vca.ERR_WORKSPACE
