@@ -21,7 +21,7 @@ for the five workloads:
 from __future__ import annotations
 
 import math
-from dataclasses import dataclass, field, replace
+from dataclasses import dataclass, replace
 
 import torch
 

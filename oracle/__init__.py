@@ -20,7 +20,6 @@ passage and the reading taken where the pages are silent.
 from __future__ import annotations
 
 import ctypes
-import os
 
 import numpy as np
 

@@ -1,4 +1,4 @@
-"""Shared helpers for the parity tests: input generation, oracle runs, metrics."""
+"""Shared helpers for the parity tests: bf16 bit patterns, row sampling, metrics."""
 from __future__ import annotations
 
 import math
@@ -6,7 +6,6 @@ import math
 import numpy as np
 import torch
 
-import oracle
 from bit_attention_video_02_b200 import workloads as W
 
 

@@ -8,7 +8,6 @@ Kept in a file that pytest collects last; it passes alone in a fresh process
 and after the rest of the suite."""
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
