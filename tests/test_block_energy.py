@@ -91,3 +91,32 @@ def test_sorting_by_clusters_raises_the_share():
     Vp = V[:, :, perm]
     same = bench.block_mean_energy(Vp, torch.arange(N).reshape(1, 1, N), None)
     assert same["sequence"] == pytest.approx(got["sorted"], abs=1e-4)
+
+
+def test_kmeans_order_reaches_the_between_cluster_share_on_a_separable_mixture():
+    # 8 well-separated clusters of exactly 128 tokens in shuffled order, one of
+    # them at each k-means seed position (token c*N/k): the grouping must recover
+    # the clusters, every sorted block is one cluster, and the share equals the
+    # between-cluster energy fraction sum_c n_c |mean_c|^2 / sum |v|^2
+    rng = np.random.default_rng(5)
+    N, d, k = 1024, 128, 8
+    lab = rng.permutation(np.repeat(np.arange(k), N // k))
+    for c in range(k):                      # cluster c at seed position c * 128
+        j = np.flatnonzero(lab == c)[0]
+        lab[[j, c * 128]] = lab[[c * 128, j]]
+    cent = rng.standard_normal((k, d)) * 4
+    v = (cent[lab] + 0.05 * rng.standard_normal((N, d))).astype(np.float32)
+    vb = torch.from_numpy(v).to(torch.bfloat16)
+    vbits = vb.view(torch.int16).numpy().view(np.uint16)
+    cents, assign, counts = oracle.kmeans_head(vbits, k, 3)
+    perm = oracle.stable_perm(assign, k)
+    # the partition is recovered (cluster ids may be relabelled)
+    assert sorted(counts.tolist()) == [128] * k
+    for c in range(k):
+        assert len(np.unique(assign[lab == c])) == 1
+    vf = vb.float().numpy().astype(np.float64)
+    between = sum(128 * float((vf[lab == c].mean(axis=0) ** 2).sum()) for c in range(k)) / float((vf ** 2).sum())
+    got = bench.block_mean_energy(vb.float().reshape(1, 1, N, d), torch.from_numpy(perm.astype(np.int64)).reshape(1, 1, N),
+                                  None)
+    assert got["sorted"] == pytest.approx(between, abs=1e-4)
+    assert got["sequence"] < 0.5 * between
