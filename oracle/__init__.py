@@ -73,6 +73,7 @@ def _declare(L):
     L.vo_smooth_quantize_head.argtypes = [vp] * 4 + [i32, i32] + [vp] * 7
     L.vo_attention_head.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, vp, vp, vp]
     L.vo_attention_head_bf16.argtypes = [vp] * 4 + [i32, i32, f64, vp, i32, i32, vp]
+    L.vo_smooth_quantize_head_vhead.argtypes = [vp] * 4 + [i32, i32] + [vp] * 7
     L.vo_sage_quantize_head.argtypes = [vp] * 3 + [i32, i32] + [vp] * 7
     L.vo_attention_head_sage.argtypes = [vp] * 6 + [i32, i32, f64, vp, i32, i32, vp, vp]
     L.vo_attention_head_skip.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, f64, vp, vp, vp]
@@ -189,8 +190,9 @@ def v_exponent(amax: float) -> int:
     return int(lib().vo_v_exponent(float(amax)))
 
 
-def smooth_quantize_head(Q, K, V, perm):
-    """One head of V-Smooth prep; inputs [N, d] uint16 bf16 bits, perm [N] int32."""
+def smooth_quantize_head(Q, K, V, perm, v_scale: str = "block"):
+    """One head of V-Smooth prep; inputs [N, d] uint16 bf16 bits, perm [N] int32.
+    v_scale "block" (one V residual exponent per block) or "head" (one per head)."""
     Q, K, V = (np.ascontiguousarray(a, dtype=np.uint16) for a in (Q, K, V))
     perm = np.ascontiguousarray(perm, dtype=np.int32)
     N, d = Q.shape
@@ -201,7 +203,9 @@ def smooth_quantize_head(Q, K, V, perm):
         Kq=np.zeros((Np, d), np.uint8), k_scale=np.empty(nb, np.float32),
         VrT=np.zeros((d, Np), np.uint8), v_exp=np.empty(nb, np.int8),
         v_mean=np.empty((nb, d), np.uint16))
-    lib().vo_smooth_quantize_head(
+    assert v_scale in ("block", "head")
+    fn = lib().vo_smooth_quantize_head if v_scale == "block" else lib().vo_smooth_quantize_head_vhead
+    fn(
         _p(Q), _p(K), _p(V), _p(perm), N, d, _p(out["Qq"]), _p(out["q_scale"]),
         _p(out["Kq"]), _p(out["k_scale"]), _p(out["VrT"]), _p(out["v_exp"]),
         _p(out["v_mean"]))

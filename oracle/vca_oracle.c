@@ -387,6 +387,53 @@ void vo_smooth_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_
     }
 }
 
+/* A second reading of the V residual scale: one power-of-two exponent per head
+ * (the smallest e with max|r| <= 448 * 2^e over the whole head) instead of one
+ * per block.  E4M3 carries its own exponent, so coding every block with the
+ * head's step changes only the elements that fall below the normal range.  Same
+ * outputs as vo_smooth_quantize_head; v_exp[b] holds the head exponent for
+ * every block. */
+void vo_smooth_quantize_head_vhead(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                   const int32_t* perm, int N, int d,
+                                   uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                                   uint8_t* VrT, int8_t* v_exp, uint16_t* v_mean) {
+    int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    int64_t Np = (int64_t)nb * VO_BLOCK;
+    float* R = (float*)malloc((size_t)N * d * sizeof(float));   /* residuals, permuted order */
+    float* bmax = (float*)malloc((size_t)nb * sizeof(float));
+    memset(VrT, 0, (size_t)d * Np);
+#pragma omp parallel for schedule(dynamic)
+    for (int b = 0; b < nb; ++b) {
+        int n0 = b * VO_BLOCK;
+        int nv = N - n0 < VO_BLOCK ? N - n0 : VO_BLOCK;
+        float* xq = (float*)malloc((size_t)VO_BLOCK * d * sizeof(float));
+        float* xk = (float*)malloc((size_t)VO_BLOCK * d * sizeof(float));
+        for (int t = 0; t < nv; ++t) {
+            int64_t src = perm[n0 + t];
+            for (int c = 0; c < d; ++c) {
+                xq[t * d + c] = vo_bf16_to_float(Q[(int64_t)(n0 + t) * d + c]);
+                xk[t * d + c] = vo_bf16_to_float(K[src * d + c]);
+                R[(int64_t)(n0 + t) * d + c] = vo_bf16_to_float(V[src * d + c]);
+            }
+        }
+        quant_rows_block(xq, nv, d, Qq + (int64_t)n0 * d, &q_scale[b]);
+        quant_rows_block(xk, nv, d, Kq + (int64_t)n0 * d, &k_scale[b]);
+        bmax[b] = v_block_residual(R + (int64_t)n0 * d, nv, d, v_mean + (int64_t)b * d);
+        free(xq); free(xk);
+    }
+    float amax = 0.0f;
+    for (int b = 0; b < nb; ++b)
+        if (bmax[b] > amax) amax = bmax[b];
+    int e = vo_v_exponent(amax);
+    for (int b = 0; b < nb; ++b) v_exp[b] = (int8_t)e;
+#pragma omp parallel for schedule(static)
+    for (int c = 0; c < d; ++c)
+        for (int j = 0; j < N; ++j)
+            VrT[(int64_t)c * Np + j] = vo_e4m3_encode(ldexpf(R[(int64_t)j * d + c], -e));
+    free(R);
+    free(bmax);
+}
+
 /* The 4-bit V-Smooth variant ([VCA-mtp] abstract and Chinese section: a 4-bit
  * V-Smooth runs on workstation cards; ExpCast is 8-bit only because NVFP4 has
  * no single affine log-to-code map).  READING: the 4-bit change is confined to

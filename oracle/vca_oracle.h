@@ -118,6 +118,13 @@ void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8
                             int N, int d, double softmax_scale, const int32_t* rows, int nrows,
                             int flags, double* O, double* lse);
 
+/* A second reading of the V residual scale: one exponent per head (v_exp[b] all
+ * equal to it); everything else as vo_smooth_quantize_head. */
+void vo_smooth_quantize_head_vhead(const uint16_t* Q, const uint16_t* K, const uint16_t* V,
+                                   const int32_t* perm, int N, int d,
+                                   uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                                   uint8_t* VrT, int8_t* v_exp, uint16_t* v_mean);
+
 /* The 4-bit V-Smooth variant ("Nunchux AI Introduces VC-Attention...",
  * abstract: 4-bit V-Smooth on workstation cards; ExpCast is 8-bit only).
  * Q, K, v_mean as in vo_smooth_quantize_head; the V residual in NVFP4:

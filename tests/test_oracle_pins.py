@@ -330,6 +330,55 @@ def test_quantize_v_reconstruction_bound(N):
         assert np.all(np.abs(mu - exact) <= np.abs(exact) * 2 ** -8 + 1e-30)
 
 
+@pytest.mark.parametrize("N", [1, 700])
+def test_quantize_v_per_head_exponent_reading(N):
+    # the second reading: one V exponent per head.  Q, K and the means are the
+    # per-block prep's; the head exponent is the largest block exponent (the
+    # exponent rule is monotone in max|r|); every residual is within half an
+    # E4M3 step of the head's scale
+    rng = np.random.default_rng(N)
+    Q, K, _ = _head(N, scale=2.0)
+    # blocks whose residuals differ by octaves
+    V = bf16_bits_of(rng.standard_normal((N, 128)) * np.exp2(np.arange(N) // 128 % 5 - 2)[:, None])
+    perm = np.arange(N, dtype=np.int32)
+    blk = oracle.smooth_quantize_head(Q, K, V, perm)
+    hd = oracle.smooth_quantize_head(Q, K, V, perm, v_scale="head")
+    for key in ("Qq", "q_scale", "Kq", "k_scale", "v_mean"):
+        assert np.array_equal(blk[key], hd[key]), key
+    e = int(blk["v_exp"].max())
+    assert np.all(hd["v_exp"] == e)
+    vf = bits_to_f32(V).astype(np.float64)
+    mu = bits_to_f32(hd["v_mean"]).astype(np.float64)[np.arange(N) // 128]
+    r = vf - mu
+    rh = oracle.e4m3_decode_table()[hd["VrT"][:, :N].T] * 2.0 ** e
+    y = np.abs(r) / 2.0 ** e
+    step = np.exp2(np.maximum(np.floor(np.log2(np.maximum(y, 1e-300))), -6) - 3)
+    assert np.all(np.abs(rh - r) <= 0.5 * step * 2.0 ** e + 1e-12)
+    # the blocks that already had the head's exponent are coded identically
+    nb = (N + 127) // 128
+    for b in range(nb):
+        if blk["v_exp"][b] == e:
+            assert np.array_equal(blk["VrT"][:, b * 128:(b + 1) * 128], hd["VrT"][:, b * 128:(b + 1) * 128])
+
+
+def test_per_head_exponent_changes_attention_little():
+    # the two readings of the V scale give nearly the same attention: E4M3's own
+    # exponent absorbs the spread of the block exponents (measured 3e-7 .. 2e-6
+    # relative on the synthetic workloads; bounded here at 1e-4)
+    from bit_attention_video_02_b200 import workloads as W
+    w = W.shrink(W.WORKLOADS[1], H=1)
+    Q, K, V = W.make_qkv(w, "cpu")
+    q, k, v = (W.bf16_bits(t[0, 0]) for t in (Q, K, V))
+    ops = oracle.prep_head(q, k, v, w.k, 3)
+    hd = oracle.smooth_quantize_head(q, k, v, ops["perm"], v_scale="head")
+    rows = np.arange(0, w.N, 7, dtype=np.int32)
+    sc = 1 / np.sqrt(128)
+    o_blk, _, _ = oracle.attention_head(ops, w.N, sc, rows)
+    o_hd, _, _ = oracle.attention_head(hd, w.N, sc, rows)
+    assert np.linalg.norm(o_hd - o_blk) / np.linalg.norm(o_blk) < 1e-4
+    assert not np.array_equal(hd["VrT"], ops["VrT"])
+
+
 # ----------------------------------------------------------------- attention
 def _bits(rng, N, s=1.0):
     return bf16_bits_of(rng.standard_normal((N, 128)) * s)
