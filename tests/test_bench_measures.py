@@ -1,7 +1,8 @@
-"""The block-mean energy measurement of bench.py (CPU): the share of a head's
-value energy that its 128-token block means carry, in sequence order, in
-static cubes of the latent grid and in k-means order ("Nunchux AI Introduces
-VC-Attention ...", abstract: 8 % / 12 % / 36 % on Wan2.2 heads)."""
+"""CPU checks of measurements bench.py reports: the block-mean energy share
+(the share of a head's value energy that its 128-token block means carry, in
+sequence order, in static cubes of the latent grid and in k-means order;
+"Nunchux AI Introduces VC-Attention ...", abstract: 8 % / 12 % / 36 % on
+Wan2.2 heads) and the algorithmic byte counts behind the roofline fractions."""
 import os
 import sys
 
@@ -120,3 +121,18 @@ def test_kmeans_order_reaches_the_between_cluster_share_on_a_separable_mixture()
                                   None)
     assert got["sorted"] == pytest.approx(between, abs=1e-4)
     assert got["sequence"] < 0.5 * between
+
+
+def test_roofline_byte_counts_match_their_closed_forms():
+    # the algorithmic bytes the bench divides by, per (b, h), as stated beside the kernels
+    from bit_attention_video_02_b200 import workloads as W
+    w = W.WORKLOADS[3]
+    N, d, nb = w.N, w.d, (w.N + 127) // 128
+    Np = 128 * nb
+    per_head = 3 * N * d * 2 + 4 * N + 2 * Np * d + Np * 64 + Np * 8 + 2 * nb * 4 + nb * d * 2 + 4
+    assert bench.fp4_prep_algorithmic_bytes(w) == w.B * w.H * per_head == 3_333_270_880
+    # 8-bit prep: Q, K, V in once and Qq, Kq, VrT out (9 B per element), V once more per
+    # k-means round, the block means
+    assert bench.prep_algorithmic_bytes(w) == 9.0 * w.B * w.H * N * d + 3 * 2.0 * w.B * w.H * N * d \
+        + 2.0 * w.B * w.H * nb * d
+    assert bench.whole_job_value(2, w.flops, 0.1) == pytest.approx(2 * w.flops / 0.1 / 1e12)
