@@ -15,6 +15,10 @@
  *              abstract).
  *   [VCA-ru]   "VC-Attention" (aikraft.ru news), section "Решение:
  *              VC-Attention без дообучения".
+ *   [TRT-blog] "Accelerating Video Generation with GEMM Quantization, Attention
+ *              Quantization and Skip Softmax Attention in TensorRT-LLM": the
+ *              Skip Softmax rule, the SAGE-style comparison recipe and the NVFP4
+ *              format (E2M1 elements, E4M3 scale per 16, fp32 per tensor).
  *
  * Arithmetic: fp64 wherever the method does not fix a precision; fp32 with
  * explicit fmaf() where the method (or a stated reading of it) fixes fp32.
