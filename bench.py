@@ -380,11 +380,15 @@ def run_ours(args, world, rank, local):
         "skip_softmax": skip,
         "sage_comparison": sage,
         "fp8_over_bf16": round(bf16_ms / (t_attn * 1e3), 3) if bf16_ms else None,
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp8_peak_sust, 1),
-                     "unit": "TFLOP/s", "frac": round(achieved / fp8_peak_sust, 4), "traffic": traffic,
-                     "peak_source": f"{peak_kind}: bf16 sustained {peaks['bf16_tflops_sustained']} x "
-                                    f"{FP8_PER_BF16} nominal FP8/BF16",
-                     "frac_of_burst": round(achieved / fp8_peak_burst, 4)},
+        # the kernel runs at the full SM clock (see clocks), so its peak is the
+        # burst figure; the sustained one was measured at a lower clock under the
+        # power cap and is kept only as a labelled extra
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(fp8_peak_burst, 1),
+                     "unit": "TFLOP/s", "frac": round(achieved / fp8_peak_burst, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind}: bf16 burst {peaks['bf16_tflops']} x "
+                                    f"{FP8_PER_BF16} nominal FP8/BF16 (of measured)",
+                     "frac_of_sustained": round(achieved / fp8_peak_sust, 4),
+                     "frac_of_spec_4500": round(achieved / 4500.0, 4)},
         "e2e": e2e,
         "gpu_launches": launches_per_step * (args.steps),
         "clocks": clk.summary(),
@@ -420,7 +424,10 @@ def run_ours(args, world, rank, local):
     line["prep_roofline"] = {"bound": "hbm", "algorithmic_bytes": pb,
                              "achieved": round(pb / (prep_ms / 1e3) / 1e9, 1), "unit": "GB/s",
                              "peak": peaks["hbm_gbs"], "frac": round(pb / (prep_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4)}
-    return line, (Q, K, V, w)
+    # the FP8 output of the workload, for the fidelity check on the host
+    O_fp8 = vca.attention_fwd(ops, N, scale, ws=ws)
+    torch.cuda.synchronize()
+    return line, (Q, K, V, w, O_fp8)
 
 
 def group_mean_energy(v: torch.Tensor, gid: torch.Tensor, ngroups: int) -> float:
@@ -547,6 +554,27 @@ def run_oracle_baseline(w, Q, K, V, rows=8192):
     return w.flops / step_s / 1e12, oracle.num_threads(), desc, step_s
 
 
+def fidelity_vs_exact(w, Q, K, V, O, nrows=256):
+    """Cosine, PSNR and relative L2 of the FP8 path's output against exact fp64
+    softmax attention (the oracle's) on seeded sampled rows of the first and
+    last head, outside the timed region."""
+    import numpy as np
+    import oracle
+    scale = 1.0 / math.sqrt(w.d)
+    out = {}
+    for h in sorted({0, w.H - 1}):
+        rng = np.random.default_rng(500 + h)
+        rows = np.sort(rng.choice(w.N, size=min(nrows, w.N), replace=False)).astype(np.int32)
+        ex = oracle.exact_attention_head(_bits(Q[0, h]), _bits(K[0, h]), _bits(V[0, h]), scale, rows=rows)
+        g = O[0, h].float().cpu().numpy().astype(np.float64)[rows]
+        cos = float((g * ex).sum() / np.sqrt((g * g).sum() * (ex * ex).sum()))
+        mse = float(np.mean((g - ex) ** 2))
+        out[f"head{h}"] = {"rows": int(len(rows)), "cosine": round(cos, 6),
+                           "psnr_db": round(10 * math.log10(float(np.abs(ex).max()) ** 2 / mse), 2),
+                           "rel_l2": round(float(np.linalg.norm(g - ex) / np.linalg.norm(ex)), 6)}
+    return out
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args, world, rank):
     if rank != 0:
@@ -593,11 +621,12 @@ def main():
         if args.impl == "reference":
             line = run_reference(args, world, rank)
         else:
-            line, (Q, K, V, w) = run_ours(args, world, rank, local)
+            line, (Q, K, V, w, O_fp8) = run_ours(args, world, rank, local)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 v, cores, desc, _ = run_oracle_baseline(w, Q, K, V)
                 line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                                         "sample": desc}
+                line["fidelity_vs_exact_fp64"] = fidelity_vs_exact(w, Q, K, V, O_fp8)
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)
     finally:

@@ -33,6 +33,8 @@ PLANT_BETA0 = 256
 PLANT_NO_RESCALE = 512
 PLANT_NIBBLE = 1024
 PLANT_P_GROUP32 = 2048
+GLOBAL_MAX = 4096      # second reading: the reference is the snapped row maximum, fixed
+NO_HEADROOM = 8192     # codes written at the reference instead of 4 octaves above it
 P_GSCALE = 0.125   # NVFP4 tensor scale of the 4-bit variant's probabilities
 BLOCK = 128
 
@@ -77,6 +79,7 @@ def _declare(L):
     L.vo_sage_quantize_head.argtypes = [vp] * 3 + [i32, i32] + [vp] * 7
     L.vo_attention_head_sage.argtypes = [vp] * 6 + [i32, i32, f64, vp, i32, i32, vp, vp]
     L.vo_attention_head_skip.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, f64, vp, vp, vp]
+    L.vo_attention_head_ex.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, f64, vp, vp, vp, vp, vp]
     L.vo_attention_head_bf16_skip.argtypes = [vp] * 4 + [i32, i32, f64, vp, i32, i32, f64, vp]
     L.vo_e2m1_decode.restype = f64
     L.vo_e2m1_decode.argtypes = [ctypes.c_uint8]
@@ -274,6 +277,27 @@ def attention_head(ops: dict, N: int, softmax_scale: float, rows=None, flags: in
         _p(c["v_exp"]), _p(c["v_mean"]), N, d, float(softmax_scale), _p(rows),
         rows.shape[0], int(flags), float(skip_lambda), _p(O), _p(lse), _p(lblk) if lblk is not None else None)
     return O, lse, lblk
+
+
+def attention_head_codes(ops: dict, N: int, softmax_scale: float, rows=None, flags: int = 0,
+                         skip_lambda: float = 0.0):
+    """As ``attention_head``, also returning what each row coded.  Returns
+    (O, lse, lblk [nrows, nb], codes [nrows, N] uint8 in permuted key order,
+    nref [nrows, nb] int32: the reference n each block was coded against)."""
+    rows = _rows(rows, N)
+    d = ops["Qq"].shape[1]
+    nb = ops["q_scale"].shape[0]
+    O = np.empty((rows.shape[0], d), np.float64)
+    lse = np.empty(rows.shape[0], np.float64)
+    lblk = np.empty((rows.shape[0], nb), np.float64)
+    codes = np.empty((rows.shape[0], N), np.uint8)
+    nref = np.empty((rows.shape[0], nb), np.int32)
+    c = {k: np.ascontiguousarray(v) for k, v in ops.items()}
+    lib().vo_attention_head_ex(
+        _p(c["Qq"]), _p(c["q_scale"]), _p(c["Kq"]), _p(c["k_scale"]), _p(c["VrT"]),
+        _p(c["v_exp"]), _p(c["v_mean"]), N, d, float(softmax_scale), _p(rows),
+        rows.shape[0], int(flags), float(skip_lambda), _p(O), _p(lse), _p(lblk), _p(codes), _p(nref))
+    return O, lse, lblk, codes, nref
 
 
 def attention_head_bf16(Q, K, V, perm, softmax_scale: float, rows=None, flags: int = 0, skip_lambda: float = 0.0):

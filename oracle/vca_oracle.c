@@ -631,16 +631,24 @@ static void p_nvfp4_block(double* pb, int n, int flags) {
 static void attn_row(const double* q, double qs, const double* kh, const double* ks,
                      const double* rh, const int* vexp, const double* mu, int N, int d,
                      double softmax_scale, int flags, double skip_log2, double* O, double* lse,
-                     double* lblk, double* z /* scratch [N] */, double* acc /* [d] */) {
+                     double* lblk, uint8_t* codes, int32_t* nref,
+                     double* z /* scratch [N] */, double* acc /* [d] */) {
     const double log2e = 1.4426950408889634074;
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
+    double zall = -INFINITY;
     for (int j = 0; j < N; ++j) {
         double s = 0.0;
         for (int c = 0; c < d; ++c) s += q[c] * kh[(int64_t)j * d + c];
         z[j] = s * qs * ks[j] * softmax_scale * log2e;
+        if (z[j] > zall) zall = z[j];
     }
+    const double headroom = (flags & VO_NO_HEADROOM) ? 0.0 : (double)VO_HEADROOM;
     for (int c = 0; c < d; ++c) acc[c] = 0.0;
     double ltot = 0.0, n = 0.0, zrun = -INFINITY;
+    /* READING (second mode, VO_GLOBAL_MAX): the reference is the row maximum
+     * over all keys snapped to the phi grid, fixed for the whole row -- the
+     * plain form of a max-subtracted softmax, no online rescale. */
+    if (flags & VO_GLOBAL_MAX) n = ceil(zall - VO_PHI);
     for (int b = 0; b < nb; ++b) {
         int j0 = b * VO_BLOCK, j1 = j0 + VO_BLOCK < N ? j0 + VO_BLOCK : N;
         double zmax = -INFINITY;
@@ -655,10 +663,14 @@ static void attn_row(const double* q, double qs, const double* kh, const double*
         if (zmax > zrun) zrun = zmax;
         if (b > 0 && zmax - zrun < skip_log2) {
             if (lblk) lblk[b] = 0.0;
+            if (codes) memset(codes + j0, 0, (size_t)(j1 - j0));
+            if (nref) nref[b] = (int32_t)n;
             continue;
         }
         double nblk = ceil(zmax - VO_PHI);
-        if (b == 0) {
+        if (flags & VO_GLOBAL_MAX) {
+            /* the reference is fixed */
+        } else if (b == 0) {
             n = nblk;
         } else if (nblk > n + VO_LAG) {
             double sc = (flags & VO_PLANT_NO_RESCALE) ? 1.0 : exp2(n - nblk);   /* exact power of two */
@@ -674,15 +686,16 @@ static void attn_row(const double* q, double qs, const double* kh, const double*
         for (int j = j0; j < j1; ++j) {
             double p;
             if (flags & (VO_EXACT_EXP | VO_P_NVFP4)) {
-                p = exp2(z[j] - (n + VO_PHI) + VO_HEADROOM);
+                p = exp2(z[j] - (n + VO_PHI) + headroom);
             } else {
-                /* = 8(z - m) + 55.65 + 8*VO_HEADROOM with m = n + phi */
-                double x = 8.0 * z[j] + 55.0 - 8.0 * n + 8.0 * VO_HEADROOM;
+                /* = 8(z - m) + 55.65 + 8*headroom with m = n + phi */
+                double x = 8.0 * z[j] + 55.0 - 8.0 * n + 8.0 * headroom;
                 if (flags & VO_PLANT_BETA0) x += 0.35;
                 double r = (flags & VO_PLANT_TRUNC) ? floor(x) : nearbyint(x);
                 if (r < 0.0) r = 0.0;
                 if (r > 126.0) r = 126.0;
                 p = vo_e4m3_decode((uint8_t)r);
+                if (codes) codes[j] = (uint8_t)r;
             }
             pb[j - j0] = p;
         }
@@ -698,17 +711,18 @@ static void attn_row(const double* q, double qs, const double* kh, const double*
             if (!(flags & VO_PLANT_NO_MEAN)) acc[c] += lb * mu[(int64_t)b * d + c];
         }
         if (lblk) lblk[b] = lb;
+        if (nref) nref[b] = (int32_t)n;
         ltot += lb;
     }
     for (int c = 0; c < d; ++c) O[c] = acc[c] / ltot;
-    if (lse) *lse = log(2.0) * ((n + VO_PHI - VO_HEADROOM) + log2(ltot));
+    if (lse) *lse = log(2.0) * ((n + VO_PHI - headroom) + log2(ltot));
 }
 
 static void attn_rows(const double* qh, const double* qs_row, const double* kh,
                       const double* ks, const double* rh, const int* vexp,
                       const double* mu, int N, int d, double softmax_scale,
                       const int32_t* rows, int nrows, int flags, double skip_log2, double* O,
-                      double* lse, double* lblk) {
+                      double* lse, double* lblk, uint8_t* codes, int32_t* nref) {
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
 #pragma omp parallel
     {
@@ -719,7 +733,8 @@ static void attn_rows(const double* qh, const double* qs_row, const double* kh,
             int i = rows[r];
             attn_row(qh + (int64_t)i * d, qs_row[i], kh, ks, rh, vexp, mu, N, d,
                      softmax_scale, flags, skip_log2, O + (int64_t)r * d, lse ? &lse[r] : NULL,
-                     lblk ? lblk + (int64_t)r * nb : NULL, z, acc);
+                     lblk ? lblk + (int64_t)r * nb : NULL, codes ? codes + (int64_t)r * N : NULL,
+                     nref ? nref + (int64_t)r * nb : NULL, z, acc);
         }
         free(z);
         free(acc);
@@ -742,6 +757,15 @@ void vo_attention_head_skip(const uint8_t* Qq, const float* q_scale, const uint8
                             const uint16_t* v_mean, int N, int d, double softmax_scale,
                             const int32_t* rows, int nrows, int flags, double skip_lambda,
                             double* O, double* lse, double* lblk) {
+    vo_attention_head_ex(Qq, q_scale, Kq, k_scale, VrT, v_exp, v_mean, N, d, softmax_scale, rows, nrows, flags,
+                         skip_lambda, O, lse, lblk, NULL, NULL);
+}
+
+void vo_attention_head_ex(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                          const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                          const uint16_t* v_mean, int N, int d, double softmax_scale,
+                          const int32_t* rows, int nrows, int flags, double skip_lambda,
+                          double* O, double* lse, double* lblk, uint8_t* codes, int32_t* nref) {
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
     int64_t Np = (int64_t)nb * VO_BLOCK;
     double* qh = (double*)malloc((size_t)N * d * sizeof(double));
@@ -765,7 +789,7 @@ void vo_attention_head_skip(const uint8_t* Qq, const float* q_scale, const uint8
         for (int c = 0; c < d; ++c) mu[(int64_t)b * d + c] = vo_bf16_to_float(v_mean[(int64_t)b * d + c]);
     }
     attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, skip_log2_of(skip_lambda), O,
-              lse, lblk);
+              lse, lblk, codes, nref);
     free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
 }
 
@@ -794,7 +818,8 @@ void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8
             rh[(int64_t)j * d + c] = vo_e4m3_decode(VcT[(int64_t)c * Np + j]);
         }
     }
-    attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, -INFINITY, O, lse, NULL);
+    attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, -INFINITY, O, lse, NULL, NULL,
+              NULL);
     for (int r = 0; r < nrows; ++r)
         for (int c = 0; c < d; ++c) O[(int64_t)r * d + c] *= v_chscale[c];
     free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
@@ -841,7 +866,7 @@ void vo_attention_head_fp4(const uint8_t* Qq, const float* q_scale, const uint8_
     for (int b = 0; b < nb; ++b)
         for (int c = 0; c < d; ++c) mu[(int64_t)b * d + c] = vo_bf16_to_float(v_mean[(int64_t)b * d + c]);
     attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags | VO_P_NVFP4, -INFINITY, O,
-              lse, NULL);
+              lse, NULL, NULL, NULL);
     free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
 }
 
@@ -921,7 +946,7 @@ void vo_attention_head_bf16_skip(const uint16_t* Q, const uint16_t* K, const uin
         }
     }
     attn_rows(qh, ones, kh, ones, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags,
-              skip_log2_of(skip_lambda), O, NULL, NULL);
+              skip_log2_of(skip_lambda), O, NULL, NULL, NULL, NULL);
     free(qh); free(kh); free(rh); free(ones); free(mu); free(ve);
 }
 

@@ -45,6 +45,8 @@ extern "C" {
 #define VO_PLANT_NO_RESCALE 512 /* planted mistake: reference moves without rescaling */
 #define VO_PLANT_NIBBLE    1024 /* planted mistake (4-bit): V nibbles read high first  */
 #define VO_PLANT_P_GROUP32 2048 /* planted mistake (4-bit): P groups of 32 keys       */
+#define VO_GLOBAL_MAX      4096 /* second reading: fixed reference = snapped row max  */
+#define VO_NO_HEADROOM     8192 /* codes written at the reference (no 4-octave pre-scale) */
 
 /* E4M3 (OCP FP8: 1 sign, 4 exponent bits with bias 7, 3 mantissa bits,
  * no infinities, NaN = S.1111.111, largest finite 448). */
@@ -109,6 +111,16 @@ void vo_attention_head_skip(const uint8_t* Qq, const float* q_scale, const uint8
                             const uint16_t* v_mean, int N, int d, double softmax_scale,
                             const int32_t* rows, int nrows, int flags, double skip_lambda,
                             double* O, double* lse, double* lblk);
+
+/* Same, also returning what each row coded: codes [nrows][N] (the E4M3 byte
+ * written for each permuted key, against the reference in effect when its
+ * block was visited; 0 for dropped blocks) and nref [nrows][nb] (that
+ * reference's integer n, the maximum being n + 0.65/8).  Both nullable. */
+void vo_attention_head_ex(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                          const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
+                          const uint16_t* v_mean, int N, int d, double softmax_scale,
+                          const int32_t* rows, int nrows, int flags, double skip_lambda,
+                          double* O, double* lse, double* lblk, uint8_t* codes, int32_t* nref);
 
 /* SAGE-style comparison recipe (TensorRT-LLM video post, section "Quantized
  * Attention": per-token Q scales, one K scale per 16 tokens after K-mean

@@ -12,7 +12,7 @@ import torch
 import oracle
 from bit_attention_video_02_b200 import vca
 from bit_attention_video_02_b200 import workloads as W
-from helpers import bf16_to_f64, bits, cosine, psnr, rel_l2, sample_rows
+from helpers import bf16_to_f64, bits, cosine, lse_tolerance, psnr, rel_l2, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +28,35 @@ def _ids(c):
     return f"cfg{c[0]}-H{c[1] or 'full'}-N{c[2] or 'full'}"
 
 
-def _run_case(w, Q, K, V, heads, nrows, seed, want_exact=True):
+def _check_head(g, gl, ref, N, rows, scale, Qb, Kb, Vb, want_exact=True, report_global=False):
+    """One head's sampled rows: the GPU output g [rows, d] and lse gl against
+    the oracle's same-algorithm result (per-head rel-L2 <= 1e-2; lse within the
+    per-row bound that code rounding flips allow) and against exact fp64
+    attention (cosine >= 0.99, PSNR reported).  Returns a report line."""
+    o_ref, lse_ref, lblk, codes, nref = oracle.attention_head_codes(ref, N, scale, rows=rows)
+    assert np.all(np.isfinite(g))
+    tol = lse_tolerance(ref, N, rows, scale, codes, nref, lblk, lse_ref)
+    r = rel_l2(g, o_ref)
+    dl = np.abs(gl - lse_ref)
+    line = dict(rows=len(rows), rel_l2=round(r, 6), lse_maxdiff=float(dl.max()),
+                lse_tol_min=float(tol.min()), lse_over=int((dl > tol).sum()))
+    if want_exact:
+        ex = oracle.exact_attention_head(Qb, Kb, Vb, scale, rows=rows)
+        line.update(cos=round(cosine(g, ex), 6), psnr=round(psnr(g, ex), 2),
+                    oracle_rel_exact=round(rel_l2(o_ref, ex), 6), gpu_rel_exact=round(rel_l2(g, ex), 6))
+    if report_global:
+        # the second reading: reference fixed at the snapped row maximum
+        og, _, _ = oracle.attention_head(ref, N, scale, rows=rows, flags=oracle.GLOBAL_MAX)
+        line.update(gpu_rel_globalmax=round(rel_l2(g, og), 6), online_rel_globalmax=round(rel_l2(o_ref, og), 6))
+    print(line)
+    assert r <= TOL_REL_L2, line
+    assert np.all(dl <= tol), line
+    if want_exact:
+        assert line["cos"] >= MIN_COSINE, line
+    return line
+
+
+def _run_case(w, Q, K, V, heads, nrows, seed, want_exact=True, report_global=False):
     scale = 1.0 / math.sqrt(w.d)
     ws = vca.Workspace(vca.lib().vca_cluster_permute_workspace_size(1, w.H, w.N, w.k))
     cent, assign, perm = vca.cluster_permute(V, w.k, iters=3, ws=ws)
@@ -37,36 +65,15 @@ def _run_case(w, Q, K, V, heads, nrows, seed, want_exact=True):
     torch.cuda.synchronize()
     ws.check()     # no device-side error (timeout, non-finite input) was recorded
     report = []
-    gs, os_, es = [], [], []
     for h in heads:
         rows = sample_rows(w.N, nrows, seed + h) if nrows else np.arange(w.N, dtype=np.int32)
         Qb, Kb, Vb = (bits(t[0, h]) for t in (Q, K, V))
         ref = oracle.prep_head(Qb, Kb, Vb, w.k, 3)
-        o_ref, lse_ref, _ = oracle.attention_head(ref, w.N, scale, rows=rows)
+        assert np.array_equal(perm[0, h].cpu().numpy(), ref["perm"])
         g = bf16_to_f64(O[0, h])[rows]
         gl = lse[0, h].cpu().numpy().astype(np.float64)[rows]
-        assert np.all(np.isfinite(g))
-        gs.append(g)
-        os_.append(o_ref)
-        r = rel_l2(g, o_ref)
-        line = dict(head=h, rows=len(rows), rel_l2=r, lse_maxdiff=float(np.abs(gl - lse_ref).max()))
-        if want_exact:
-            ex = oracle.exact_attention_head(Qb, Kb, Vb, scale, rows=rows)
-            es.append(ex)
-            line.update(cos=cosine(g, ex), psnr=psnr(g, ex), ref_rel_exact=rel_l2(o_ref, ex))
-        report.append(line)
-    g = np.concatenate(gs)
-    o = np.concatenate(os_)
-    for line in report:
-        print(line)
-    assert rel_l2(g, o) <= TOL_REL_L2, report
-    # lse agrees with the oracle's (log of the decoded row sum at the reference
-    # max); a code that rounds the other way at an fp32-vs-fp64 boundary moves
-    # one probability by at most one E4M3 step (1/8), so rows dominated by a
-    # few keys can differ by a few 1e-3
-    assert max(l["lse_maxdiff"] for l in report) < 5e-3, report
-    if want_exact:
-        assert cosine(g, np.concatenate(es)) >= MIN_COSINE, report
+        line = _check_head(g, gl, ref, w.N, rows, scale, Qb, Kb, Vb, want_exact, report_global)
+        report.append(dict(head=h, **line))
     return report
 
 
@@ -78,36 +85,54 @@ def test_attention_matches_oracle(case):
     _run_case(w, Q, K, V, range(w.H), nrows, seed=cid)
 
 
+def _spread_heads(H):
+    return sorted({0, H // 3, (2 * H) // 3, H - 1})
+
+
 @pytest.mark.parametrize("cid", [3, 5])
 def test_attention_full_size_sampled_rows(cid):
-    # the benchmark's launch configuration (all heads, full N), checked on
-    # sampled rows of the first and last head
+    # the benchmark's launch configuration (all heads, full N), checked on 256
+    # sampled rows of four heads spread over the layer, first and last included
     w = W.WORKLOADS[cid]
     Q, K, V = W.make_qkv(w, "cuda")
-    _run_case(w, Q, K, V, (0, w.H - 1), 48, seed=100 + cid)
+    _run_case(w, Q, K, V, _spread_heads(w.H), 256, seed=100 + cid, report_global=True)
 
 
-def test_attention_denoising_steps_reuse_permutation():
-    # permutation computed at step 0, reused at steps 1..3 (fidelity per step)
-    w = W.shrink(W.WORKLOADS[4], H=2, N=2048)
+def test_attention_denoising_steps_full_size():
+    # the denoising-step workload at full size (H=24, N=32768): the permutation
+    # is computed at step 0 and reused at steps 1..3; every step is checked on
+    # 256 sampled rows of four heads, with cosine and PSNR against exact fp64
+    # attention reported per step
+    w = W.WORKLOADS[4]
     scale = 1.0 / math.sqrt(w.d)
+    heads = _spread_heads(w.H)
     Q0, K0, V0 = W.make_qkv(w, "cuda", step=0)
-    _, _, perm0 = vca.cluster_permute(V0, w.k, iters=3)
+    ws = vca.Workspace(vca.lib().vca_cluster_permute_workspace_size(1, w.H, w.N, w.k))
+    _, _, perm0 = vca.cluster_permute(V0, w.k, 3, ws=ws)
+    torch.cuda.synchronize()
+    ref_perm = {}
+    for h in heads:
+        ref0 = oracle.prep_head(bits(Q0[0, h]), bits(K0[0, h]), bits(V0[0, h]), w.k, 3)
+        assert np.array_equal(perm0[0, h].cpu().numpy(), ref0["perm"])
+        ref_perm[h] = ref0["perm"]
+    del Q0, K0, V0
     for step in range(4):
         Q, K, V = W.make_qkv(w, "cuda", step=step)
-        ops = vca.smooth_quantize(Q, K, V, perm0)
-        O = vca.attention_fwd(ops, w.N, scale)
+        ops = vca.smooth_quantize(Q, K, V, perm0, ws=ws)
+        O, lse = vca.attention_fwd(ops, w.N, scale, want_lse=True, ws=ws)
         torch.cuda.synchronize()
-        for h in range(w.H):
+        ws.check()
+        for h in heads:
             Qb, Kb, Vb = (bits(t[0, h]) for t in (Q, K, V))
-            ref = oracle.smooth_quantize_head(Qb, Kb, Vb, perm0[0, h].cpu().numpy())
-            rows = sample_rows(w.N, 256, step * 10 + h)
-            o_ref, _, _ = oracle.attention_head(ref, w.N, scale, rows=rows)
+            ref = oracle.smooth_quantize_head(Qb, Kb, Vb, ref_perm[h])
+            for name in ("Qq", "Kq", "VrT", "v_exp"):
+                assert np.array_equal(ops[name][0, h].cpu().numpy(), ref[name]), (step, h, name)
+            rows = sample_rows(w.N, 256, 400 + 10 * step + h)
             g = bf16_to_f64(O[0, h])[rows]
-            ex = oracle.exact_attention_head(Qb, Kb, Vb, scale, rows=rows)
-            print(dict(step=step, head=h, rel_l2=rel_l2(g, o_ref), cos=cosine(g, ex), psnr=psnr(g, ex)))
-            assert rel_l2(g, o_ref) <= TOL_REL_L2
-            assert cosine(g, ex) >= MIN_COSINE
+            gl = lse[0, h].cpu().numpy().astype(np.float64)[rows]
+            line = _check_head(g, gl, ref, w.N, rows, scale, Qb, Kb, Vb)
+            print(dict(step=step, head=h, cos=line["cos"], psnr=line["psnr"]))
+        del Q, K, V, ops, O, lse
 
 
 def test_attention_identity_permutation_and_scale():
