@@ -10,18 +10,25 @@
 //
 // Design (sm_100a):
 //  * one CTA = two 128-row query tiles of one head (they share every K/V tile);
-//    12 warps: warp 0 TMA producer, warp 1 MMA issuer (one thread) and TMEM
-//    owner, warp 2 stages block means, warps 4-7 / 8-11 are the softmax
-//    warpgroups of query tile 0 / 1 (thread = query row = TMEM lane).
-//  * TMEM (512 columns): S0, S1 (fp32 scores), O0, O1 (fp32 accumulators).
-//  * S_t = Q_t K_j^T: tcgen05 kind::f8f6f4, operands from 128B-swizzled smem.
+//    12 warps: warp 0 TMA producer, warp 1 MMA issuer (the whole warp runs the
+//    issue loop, one elected lane issues) and TMEM owner, warp 2 stages block
+//    means, warps 4-7 / 8-11 are the softmax warpgroups of query tile 0 / 1
+//    (thread = query row = TMEM lane).
+//  * TMEM (512 columns): S (one fp32 score tile, shared by the two query
+//    tiles in turn), the P region (per tile: two 4-column UE8M0 scale vectors
+//    and 32 columns of packed E4M3 codes), O0, O1 (fp32 accumulators).
+//  * S = Q_t K_j^T: tcgen05 kind::f8f6f4, operands from 128B-swizzled smem.
+//    A softmax warpgroup releases S as soon as it has loaded its scores into
+//    registers, and the MMA warp refills it for the other tile, so the tensor
+//    core computes one tile's scores while both warpgroups compute codes: the
+//    two tiles run staggered by one QK^T, and the time per key block is the
+//    softmax's, not softmax + MMAs.  The order of issue is
+//      QK0(0) QK1(0) QK0(1) | PV0(j) QK1(j+1) PV1(j) QK0(j+2) | ...
 //  * O_t += P_t R_j * 2^e_j: kind::mxf8f6f4.block_scale with A = P_t read
 //    from tensor memory (no shared-memory round trip for the probabilities);
-//    the per-block V exponent is the UE8M0 scale of B (A's scale is 1).  P_t
-//    (32 columns of packed E4M3 codes) and the two 4-column scale vectors are
-//    written into the already-consumed S_t columns, so the next QK^T (issued
-//    after this PV; tensor-core ops run in issue order) overwrites them only
-//    after they were read.
+//    the per-block V exponent is the UE8M0 scale of B (A's scale is 1).  A
+//    warpgroup writes P_t(j) and the scale vectors only after PV_t(j-1) has
+//    completed (o_done), which it needs anyway before rescaling O_t.
 //  * Mean restore: every 8 key blocks, O_t += L_t M^T with a TF32 MMA, where
 //    L_t[i][b] are the block row sums (split hi + lo so they keep ~22 bits) and
 //    M[d][b] the bf16 block means (exact in TF32).
@@ -42,6 +49,11 @@ namespace vca {
 constexpr int kAttnThreads = 384;
 constexpr int kStages = 3;
 constexpr int kGroup = 8;   // key blocks per mean-restore MMA
+
+// TMEM columns
+constexpr uint32_t kColS = 0;     // score tile (128 columns)
+constexpr uint32_t kColP = 128;   // P region: tile t at +64t: scale vectors +0..+7, codes +8..+39
+constexpr uint32_t kColO = 256;   // O_t at +128t
 
 // dynamic shared memory layout (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                         // 2 x 16 KB
@@ -74,7 +86,8 @@ struct __align__(8) AttnBars {
   uint64_t q_full;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
+  uint64_t s_full[2];    // S holds tile t's scores of the current block
+  uint64_t s_free[2];    // tile t's warpgroup has loaded them (S may be refilled)
   uint64_t p_full[2];
   uint64_t o_done[2];
   uint64_t mu_full[2];
@@ -125,6 +138,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&bars.s_full[t], 1);
+      mbar_init(&bars.s_free[t], 128);
       mbar_init(&bars.p_full[t], 128);
       mbar_init(&bars.o_done[t], 1);
       mbar_init(&bars.mu_full[t], 32);
@@ -191,65 +205,86 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const uint64_t dL = smem_desc(smem_u32(sm + kOffL), 128, 256, kLayoutNone);
     const uint64_t dMu = smem_desc(smem_u32(sm + kOffMu), 128, 256, kLayoutNone);
     unsigned long long nskip = 0;   // Skip Softmax: PVs skipped by this CTA
+    const uint32_t tS = tmem + kColS;
+    // S <- Q_t K_jj^T (K_jj in stage jj % kStages, already waited for)
+    auto issue_qk = [&](int t, int jj) {
+      const int s1 = jj % kStages;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_f8_ss_w(tS, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(s1 * 1024 + 2 * k), id_qk, k > 0);
+      tc_commit_w(&bars.s_full[t]);
+    };
+    // O_t += P_t(j) R_j 2^e_j, and at a group end the mean restore of the group;
+    // o_done[t] then tracks everything that reads the P region or writes O_t
+    auto issue_pv = [&](int t, int j) -> bool {
+      if (!mbar_wait_warp(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t)) return false;
+      tc_fence_after();
+      const int s = j % kStages;
+      const uint32_t tP = tmem + kColP + t * 64;   // scale vectors at +0 / +4, codes at +8..+39
+      // (the flags were written before the warpgroup's p_full arrivals)
+      bool skip_pv = false;
+      if (SKIP) {
+        const volatile int* f = warp_drop_s[t];
+        skip_pv = f[0] && f[1] && f[2] && f[3];
+        nskip += skip_pv ? 1 : 0;
+      }
+      if (!skip_pv) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)   // 8 columns (32 codes) per K step
+          mma_mxf8_ts_w(tmem + kColO + t * 128, tP + 8 + 8 * k, dV + (uint64_t)(s * 1024 + 2 * k), id_pv, tP,
+                        tP + 4, (j > 0 || k > 0) ? 1u : 0u);
+      }
+      const bool group_end = (j % kGroup == kGroup - 1) || (j == nkv - 1);
+      if (group_end && !SAGE) {
+        const int g = j / kGroup, gb = g & 1;
+        if (!mbar_wait_warp(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220)) return false;
+        tc_fence_after();
+        const uint64_t bdesc = dMu + (uint64_t)(gb * 256);
+        mma_tf32_ss_w(tmem + kColO + t * 128, dL + (uint64_t)(t * 512), bdesc, id_mu, 1u);
+        mma_tf32_ss_w(tmem + kColO + t * 128, dL + (uint64_t)(t * 512 + 256), bdesc, id_mu, 1u);
+        if (t == 1) tc_commit_w(&bars.mu_empty[gb]);
+      }
+      tc_commit_w(&bars.o_done[t]);
+      return true;
+    };
     bool ok = mbar_wait_warp(&bars.q_full, 0, &abort_s, p.st, lim, 200);
     ok = ok && mbar_wait_warp(&bars.kv_full[0], 0, &abort_s, p.st, lim, 201);
     if (ok) {
       tc_fence_after();
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_f8_ss_w(tmem + t * 128, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(2 * k), id_qk, k > 0);
-        tc_commit_w(&bars.s_full[t]);
+      issue_qk(0, 0);
+    }
+    ok = ok && mbar_wait_warp(&bars.s_free[0], 0, &abort_s, p.st, lim, 202);
+    if (ok) {
+      tc_fence_after();
+      issue_qk(1, 0);
+    }
+    if (ok && nkv > 1) {
+      ok = mbar_wait_warp(&bars.s_free[1], 0, &abort_s, p.st, lim, 203) &&
+           mbar_wait_warp(&bars.kv_full[1 % kStages], (1 / kStages) & 1, &abort_s, p.st, lim, 204);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0, 1);
       }
     }
     for (int j = 0; ok && j < nkv; ++j) {
-      const int s = j % kStages;
-      const bool group_end = (j % kGroup == kGroup - 1) || (j == nkv - 1);
-      const int g = j / kGroup, gb = g & 1;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        ok = mbar_wait_warp(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t);
+      ok = issue_pv(0, j);
+      if (!ok) break;
+      if (j + 1 < nkv) {   // tile 0 has loaded S_0(j+1): S takes tile 1's scores
+        ok = mbar_wait_warp(&bars.s_free[0], (j + 1) & 1, &abort_s, p.st, lim, 230);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t sft = tmem + t * 128;   // scale vectors live in the consumed S_t columns
-        // (the flags were written before the warpgroup's p_full arrivals)
-        bool skip_pv = false;
-        if (SKIP) {
-          const volatile int* f = warp_drop_s[t];
-          skip_pv = f[0] && f[1] && f[2] && f[3];
-          nskip += skip_pv ? 1 : 0;
-        }
-        if (!skip_pv) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k)   // P_t at S_t columns 8..39, 8 columns (32 codes) per K step
-            mma_mxf8_ts_w(tmem + 256 + t * 128, sft + 8 + 8 * k, dV + (uint64_t)(s * 1024 + 2 * k), id_pv, sft,
-                          sft + 4, (j > 0 || k > 0) ? 1u : 0u);
-        }
-        if (group_end && !SAGE) {
-          ok = mbar_wait_warp(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220);
-          if (!ok) break;
-          tc_fence_after();
-          const uint64_t bdesc = dMu + (uint64_t)(gb * 256);
-          mma_tf32_ss_w(tmem + 256 + t * 128, dL + (uint64_t)(t * 512), bdesc, id_mu, 1u);
-          mma_tf32_ss_w(tmem + 256 + t * 128, dL + (uint64_t)(t * 512 + 256), bdesc, id_mu, 1u);
-          if (t == 1) tc_commit_w(&bars.mu_empty[gb]);
-        }
-        tc_commit_w(&bars.o_done[t]);
-        if (t == 1) tc_commit_w(&bars.kv_empty[s]);
-        if (j + 1 < nkv) {
-          const int s1 = (j + 1) % kStages;
-          if (t == 0) {
-            ok = mbar_wait_warp(&bars.kv_full[s1], ((j + 1) / kStages) & 1, &abort_s, p.st, lim, 230);
-            if (!ok) break;
-            tc_fence_after();
-          }
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_f8_ss_w(tmem + t * 128, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(s1 * 1024 + 2 * k),
-                        id_qk, k > 0);
-          tc_commit_w(&bars.s_full[t]);
-        }
+        issue_qk(1, j + 1);
+      }
+      ok = issue_pv(1, j);
+      if (!ok) break;
+      tc_commit_w(&bars.kv_empty[j % kStages]);   // K_j and V_j are no longer read
+      if (j + 2 < nkv) {   // tile 1 has loaded S_1(j+1): S takes tile 0's next scores
+        const int s2 = (j + 2) % kStages;
+        ok = mbar_wait_warp(&bars.s_free[1], (j + 1) & 1, &abort_s, p.st, lim, 231) &&
+             mbar_wait_warp(&bars.kv_full[s2], ((j + 2) / kStages) & 1, &abort_s, p.st, lim, 232);
+        if (!ok) break;
+        tc_fence_after();
+        issue_qk(0, j + 2);
       }
     }
     tc_commit_w(&bars.mma_done);
@@ -277,8 +312,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const int t = (warp >> 2) - 1;                 // query tile of this warpgroup
     const int r = threadIdx.x & 127;               // query row within the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + t * 128 + lane_off;
-    const uint32_t tO = tmem + 256 + t * 128 + lane_off;
+    const uint32_t tS = tmem + kColS + lane_off;
+    const uint32_t tP = tmem + kColP + t * 64 + lane_off;   // scale vectors +0..+7, codes +8..+39
+    const uint32_t tO = tmem + kColO + t * 128 + lane_off;
     const int qtile = pair * 2 + t;
     const bool qvalid = qtile < nb;
     const bool row_valid = qvalid && qtile * 128 + r < N;
@@ -335,6 +371,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         VCA_TMEM_LD32(tS + 96, (su + 96));
         tmem_ld_wait();
       }
+      // the scores are in registers: S may take the other tile's next scores
+      tc_fence_before();
+      mbar_arrive(&bars.s_free[t]);
       const int valid = min(128, N - j * 128);
       if (valid < 128) {
 #pragma unroll
@@ -380,8 +419,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         rej = j > 0 && (!row_valid || zt - zrun < p.skip_log2);
       }
       const int ntile = (int)ceilf(SAGE ? zmx - 0.08125f : __fmaf_rn(mx, cz, -0.08125f));
-      // (S_t(j) was committed after PV_t(j-1) and any mean MMA before it, so
-      // those have completed: O_t may be rescaled and sL_t rewritten now)
       float rescale = 1.0f;       // O_t and the pending row sums are scaled by this
       if (rej) {
         // a dropped block lies below the running maximum, which the reference
@@ -404,10 +441,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       const float2 c8x2 = make_float2(c8r, c8r), baddx2 = make_float2(badd, badd);
       float2 lsa = make_float2(0.0f, 0.0f), lsb = make_float2(0.0f, 0.0f);
       uint32_t pw[32];   // the row's 128 codes, 4 per word, in key order
+      // PV_t(j-1) (and the mean restore before it) must have completed before
+      // the P region, sL_t or O_t are written; it was issued when this
+      // warpgroup finished the previous block, so this wait rarely blocks
+      if (j > 0) {
+        ok = mbar_wait_warp(&bars.o_done[t], (j - 1) & 1, &abort_s, p.st, lim, 410 + t);
+        if (!ok) break;
+        tc_fence_after();
+      }
       if (warp_drop) {
         // PV may still run for the other warps' rows: these rows contribute zeros
         const uint32_t zero[32] = {};
-        VCA_TMEM_ST32(tS + 8, zero);
+        VCA_TMEM_ST32(tP + 8, zero);
       } else {
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
@@ -422,7 +467,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         lsb = __fadd2_rn(lsb, make_float2(__uint_as_float(b2 << 20), __uint_as_float(b3 << 20)));
         pw[q] = prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
       }
-      VCA_TMEM_ST32(tS + 8, pw);
+      VCA_TMEM_ST32(tP + 8, pw);
       }
       const float lsum = (lsa.x + lsa.y) + (lsb.x + lsb.y);
       const float l = lsum * 0x1p120f;
@@ -469,7 +514,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         for (int i = 0; i < 4; ++i) sf[i] = 0x7F7F7F7Fu;
 #pragma unroll
         for (int i = 4; i < 8; ++i) sf[i] = eb * 0x01010101u;
-        tmem_st8(tS, sf);
+        tmem_st8(tP, sf);
       }
       if (SKIP && lane == 0) warp_drop_s[t][warp & 3] = warp_drop ? 1 : 0;
       fence_proxy_async_smem();
