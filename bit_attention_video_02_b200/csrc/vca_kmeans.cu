@@ -175,7 +175,8 @@ __global__ void __launch_bounds__(kSegWarps * 32) km_accum_kernel(const uint16_t
                                                                  const int32_t* __restrict__ perm,
                                                                  const int* __restrict__ cstart,
                                                                  const int* __restrict__ counts,
-                                                                 long long* __restrict__ sums, int N, int k) {
+                                                                 long long* __restrict__ sums, int N, int k,
+                                                                 DevStatus* st) {
   __shared__ int cs[VCA_MAX_CLUSTERS], ce[VCA_MAX_CLUSTERS];
   const int bh = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x < k) {
@@ -196,6 +197,7 @@ __global__ void __launch_bounds__(kSegWarps * 32) km_accum_kernel(const uint16_t
   const int32_t* pb = perm + (int64_t)bh * N;
   unsigned long long* sb = reinterpret_cast<unsigned long long*>(sums + (int64_t)bh * k * 128);
   int hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
+  uint32_t magbits = 0;   // largest |v| bit pattern seen: the exact sums need |v| < 2^20
   auto flush = [&]() {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -231,6 +233,7 @@ __global__ void __launch_bounds__(kSegWarps * 32) km_accum_kernel(const uint16_t
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           int h, l;
+          magbits = max(magbits, (uint32_t)x[u][j] & 0x7FFFu);
           fix24_split(__uint_as_float((uint32_t)x[u][j] << 16), h, l);
           hi[j] += h;
           lo[j] += l;
@@ -239,6 +242,10 @@ __global__ void __launch_bounds__(kSegWarps * 32) km_accum_kernel(const uint16_t
     }
   }
   flush();
+  // bf16 exponent field >= 127 + 20: |v| >= 2^20 (all ones: inf or NaN)
+  magbits = __reduce_max_sync(0xffffffffu, magbits);
+  if (lane == 0 && magbits >= 0x4980u)
+    report(st, magbits >= 0x7F80u ? VCA_ERR_NONFINITE : VCA_ERR_INVALID, 600, bh);
 }
 
 __global__ void km_update_kernel(const long long* __restrict__ sums, const int* __restrict__ counts,
@@ -372,7 +379,7 @@ static int cluster_permute_impl(const vca_bf16* V, int B, int H, int N, int d, i
     if ((rc = check_launch("sort_scatter_kernel"))) return rc;
     if (cudaMemsetAsync(w.sums, 0, sums_bytes, s) != cudaSuccess)
       return fail(VCA_ERR_CUDA, "vca_cluster_permute: memset failed");
-    km_accum_kernel<<<g_accum, kSegWarps * 32, 0, s>>>(V, perm, w.cstart, w.counts, w.sums, N, k);
+    km_accum_kernel<<<g_accum, kSegWarps * 32, 0, s>>>(V, perm, w.cstart, w.counts, w.sums, N, k, w.st);
     if ((rc = check_launch("km_accum_kernel"))) return rc;
     km_update_kernel<<<dim3(BH, k), 128, 0, s>>>(w.sums, w.counts, cent, k);
     if ((rc = check_launch("km_update_kernel"))) return rc;
@@ -423,22 +430,15 @@ static __device__ __align__(256) unsigned char g_cluster_scratch[VCA_NOALLOC_SCR
 // The array's host-side name is only a stand-in for the symbol; the device
 // address comes from cudaGetSymbolAddress, looked up once per device with that
 // device current (the first call on each device does it).
+// The array's device address, looked up on every call (the lookup allocates
+// nothing, and after a device reset the address may differ) with the
+// caller's device current.
 static int noalloc_scratch(void** out) {
-  static std::mutex mu;
-  static void* addr[256] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail(VCA_ERR_CUDA, "vca_cluster_permute_noalloc: cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= 256) return fail(VCA_ERR_UNSUPPORTED, "vca_cluster_permute_noalloc: device %d out of range", dev);
-  std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_cluster_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(VCA_ERR_CUDA, "vca_cluster_permute_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-    addr[dev] = p;
-  }
-  *out = addr[dev];
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_cluster_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(VCA_ERR_CUDA, "vca_cluster_permute_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+  *out = p;
   return VCA_OK;
 }
 
@@ -455,9 +455,10 @@ extern "C" int vca_cluster_permute_noalloc(const vca_bf16* V, int B, int H, int 
                 B, H, N, k, need, (size_t)VCA_NOALLOC_SCRATCH_BYTES);
   void* scratch = nullptr;
   if ((rc = noalloc_scratch(&scratch))) return rc;
-  // the array keeps the previous call's contents: the status word is cleared
-  // here; the sums and counts are cleared before every k-means round and the
-  // sort tables are written in full before they are read
+  // the array keeps the previous call's contents: its status word (where the
+  // k-means kernels record out-of-range input) is cleared here; the sums and
+  // counts are cleared before every k-means round and the sort tables are
+  // written in full before they are read
   if (cudaMemsetAsync(scratch, 0, sizeof(DevStatus), (cudaStream_t)stream) != cudaSuccess)
     return fail(VCA_ERR_CUDA, "vca_cluster_permute_noalloc: cudaMemsetAsync failed");
   size_t total;

@@ -185,9 +185,19 @@ def cluster_permute_noalloc(V: torch.Tensor, k: int, iters: int = 3, init=None, 
     fixed array inside the library); the output tensors may be passed in."""
     B, H, N, d = _bhnd(V)
     dev = V.device
-    cent = centroids if centroids is not None else torch.empty(B, H, k, d, dtype=torch.float32, device=dev)
-    assign = assign if assign is not None else torch.empty(B, H, N, dtype=torch.int32, device=dev)
-    perm = perm if perm is not None else torch.empty(B, H, N, dtype=torch.int32, device=dev)
+
+    def _out(t, shape, dtype, what):
+        if t is None:
+            return torch.empty(shape, dtype=dtype, device=dev)
+        assert tuple(t.shape) == shape and t.dtype == dtype and t.device == dev and t.is_contiguous(), \
+            f"{what} must be a contiguous {dtype} tensor of shape {shape} on {dev}"
+        return t
+
+    cent = _out(centroids, (B, H, k, d), torch.float32, "centroids")
+    assign = _out(assign, (B, H, N), torch.int32, "assign")
+    perm = _out(perm, (B, H, N), torch.int32, "perm")
+    if init is not None:
+        _out(init, (B, H, k, d), torch.float32, "init")
     _check(lib().vca_cluster_permute_noalloc(_ptr(V), B, H, N, d, k, iters, _ptr(init), _ptr(cent),
                                              _ptr(assign), _ptr(perm), _stream(stream)))
     return cent, assign, perm

@@ -118,7 +118,9 @@ size_t vca_cluster_permute_workspace_size(int B, int H, int N, int k);
  *   centroids  [B][H][k][d] fp32        (out)
  *   assign     [B][H][N] int32          (out, the assignment of the last round)
  *   perm       [B][H][N] int32          (out)
- * 1 <= k <= VCA_MAX_CLUSTERS, 1 <= iters <= 64, |V| < 2^20. */
+ * 1 <= k <= VCA_MAX_CLUSTERS, 1 <= iters <= 64, |V| < 2^20: a value outside
+ * that range records VCA_ERR_INVALID (VCA_ERR_NONFINITE for inf/NaN) in the
+ * workspace status word (vca_check_status). */
 int vca_cluster_permute(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
                         const float* init_centroids, float* centroids, int32_t* assign,
                         int32_t* perm, void* ws, size_t ws_bytes, vca_stream_t stream);
@@ -132,12 +134,15 @@ int vca_cluster_permute(const vca_bf16* V, int B, int H, int N, int d, int k, in
  * held on every GPU that loads the library until the process exits.
  *  - Shapes whose workspace (vca_cluster_permute_workspace_size) exceeds that
  *    size are rejected with VCA_ERR_UNSUPPORTED; nothing is allocated, ever.
- *  - The first call on each device looks up the array's device address (with
- *    that device current); make that first call before any stream capture.
+ *  - Every call looks up the array's device address with the caller's device
+ *    current (a lookup, no allocation).
  *  - Every call uses the same array: calls whose work overlaps on the GPU race.
  *    Issue them on one stream, or serialise them.
- *  - Device-side errors are recorded in the array's own status word and are not
- *    reported to the caller. */
+ *  - The return value reports argument and launch errors only.  The input
+ *    check the kernels make on the device (|V| >= 2^20 or non-finite values,
+ *    which the exact sums cannot take) lands in a status word inside the array
+ *    that no call returns: validate V beforehand, or use vca_cluster_permute,
+ *    whose workspace status vca_check_status reads. */
 #define VCA_NOALLOC_SCRATCH_BYTES (8u << 20)
 int vca_cluster_permute_noalloc(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
                                 const float* init_centroids, float* centroids, int32_t* assign,

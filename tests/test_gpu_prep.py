@@ -99,3 +99,21 @@ def test_nonfinite_input_is_reported():
         ws.check()
     assert e.value.code == vca.ERR_NONFINITE
     ws.check()   # cleared after reading
+
+
+@pytest.mark.parametrize("bad,code", [(2.0 ** 21, "ERR_INVALID"), (float("inf"), "ERR_NONFINITE")])
+def test_grouping_reports_values_outside_its_exact_range(bad, code):
+    # the k-means sums are exact only for |v| < 2^20: a larger or non-finite
+    # value is recorded in the workspace status word
+    w = W.shrink(W.WORKLOADS[1], H=2, N=600)
+    _, _, V = W.make_qkv(w, "cuda")
+    V[0, 1, 77, 5] = bad
+    ws = vca.Workspace(vca.lib().vca_cluster_permute_workspace_size(1, w.H, w.N, w.k))
+    vca.cluster_permute(V, w.k, 3, ws=ws)
+    with pytest.raises(vca.VcaError) as e:
+        ws.check()
+    assert e.value.code == getattr(vca, code)
+    # in range: no error
+    V[0, 1, 77, 5] = 2.0 ** 19
+    vca.cluster_permute(V, w.k, 3, ws=ws)
+    ws.check()

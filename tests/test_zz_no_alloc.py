@@ -55,3 +55,25 @@ def test_noalloc_rejects_shapes_beyond_its_fixed_scratch():
         ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(out.data_ptr()), None)
     assert rc == vca.ERR_UNSUPPORTED
     assert b"scratch" in vca.lib().vca_last_error()
+
+
+def test_noalloc_python_wrapper_matches_and_checks_its_outputs():
+    # the binding's wrapper: the same results as the workspace entry point,
+    # into caller-provided outputs; outputs of the wrong shape, dtype or device
+    # are refused before anything reaches the library
+    w = W.shrink(W.WORKLOADS[2], H=2, N=900)
+    _, _, V = W.make_qkv(w, "cuda")
+    cent = torch.empty(1, w.H, w.k, 128, dtype=torch.float32, device="cuda")
+    got = vca.cluster_permute_noalloc(V, w.k, 3, centroids=cent)
+    ref = vca.cluster_permute(V, w.k, 3)
+    torch.cuda.synchronize()
+    assert got[0] is cent
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+    bad = torch.empty(1, w.H, w.N + 1, dtype=torch.int32, device="cuda")
+    with pytest.raises(AssertionError):
+        vca.cluster_permute_noalloc(V, w.k, 3, perm=bad)
+    with pytest.raises(AssertionError):
+        vca.cluster_permute_noalloc(V, w.k, 3, assign=torch.empty(1, w.H, w.N, dtype=torch.int64, device="cuda"))
+    with pytest.raises(AssertionError):
+        vca.cluster_permute_noalloc(V, w.k, 3, init=torch.empty(1, w.H, w.k, 128, dtype=torch.float32))
