@@ -36,6 +36,7 @@ EXPORTED = [
     "vca_attention_fwd_skip", "vca_vc_attention_host_buffer_size", "vca_vc_attention_host",
     "vca_sage_quantize_workspace_size", "vca_sage_quantize_qkv", "vca_attention_fwd_sage",
     "vca_smooth_quantize_fp4_workspace_size", "vca_smooth_quantize_qkv_fp4",
+    "vca_attention_fwd_fp4", "vca_debug_fp4_mma",
 ]
 
 
@@ -82,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.vca_smooth_quantize_fp4_workspace_size.restype = sz
         L.vca_smooth_quantize_fp4_workspace_size.argtypes = [i32, i32, i32]
         L.vca_smooth_quantize_qkv_fp4.argtypes = [vp] * 4 + [i32] * 4 + [vp] * 8 + [vp, sz, vp]
+        L.vca_attention_fwd_fp4.argtypes = [vp] * 8 + [i32, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+        L.vca_debug_fp4_mma.argtypes = [vp] * 6
         L.vca_vc_attention_host_buffer_size.restype = sz
         L.vca_vc_attention_host_buffer_size.argtypes = [i32] * 6
         L.vca_vc_attention_host.argtypes = [vp, vp, vp] + [i32] * 6 + [f32, vp, i32, vp, sz, vp]
@@ -408,6 +411,39 @@ def sage_quantize(Q, K, V, ws: Workspace | None = None, stream=None) -> dict:
         _ptr(out["k_scale"]), _ptr(out["VcT"]), _ptr(out["v_chscale"]), _ptr(out["k_mean"]), ws.ptr, ws.nbytes,
         _stream(stream)))
     return out
+
+
+def attention_fwd_fp4(ops: dict, N: int, softmax_scale: float | None = None, O=None, lse=None,
+                      want_lse: bool = False, ws: Workspace | None = None, stream=None):
+    """vca_attention_fwd_fp4: attention of the 4-bit variant on the operands of
+    ``smooth_quantize_fp4`` (NVFP4 probabilities and V residual in PV)."""
+    B, H, Np, d = ops["Qq"].shape
+    scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
+    dev = ops["Qq"].device
+    if O is None:
+        O = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    need = lib().vca_attention_workspace_size(B, H, N)
+    ws = (ws or Workspace(need, dev)).ensure(need)
+    _check(lib().vca_attention_fwd_fp4(
+        _ptr(ops["Qq"]), _ptr(ops["q_scale"]), _ptr(ops["Kq"]), _ptr(ops["k_scale"]), _ptr(ops["VrT4"]),
+        _ptr(ops["v_sc"]), _ptr(ops["v_gscale"]), _ptr(ops["v_mean"]), B, H, N, d, scale, _ptr(O), _ptr(lse),
+        ws.ptr, ws.nbytes, _stream(stream)))
+    return (O, lse) if want_lse else O
+
+
+def debug_fp4_mma(a_codes, sf_cols, b_codes, ws: Workspace | None = None, stream=None) -> torch.Tensor:
+    """vca_debug_fp4_mma: one 128x128x128 block-scaled FP4 product with known
+    operands (uint8 device tensors [128, 64] A codes, [128, 64] the 16 scale
+    columns of every tensor-memory lane, [128, 64] B^T codes)."""
+    for t in (a_codes, sf_cols, b_codes):
+        assert t.is_cuda and t.dtype == torch.uint8 and tuple(t.shape) == (128, 64) and t.is_contiguous()
+    D = torch.empty(128, 128, dtype=torch.float32, device=a_codes.device)
+    ws = ws or Workspace(256, a_codes.device)
+    _check(lib().vca_debug_fp4_mma(_ptr(a_codes), _ptr(sf_cols), _ptr(b_codes), _ptr(D), ws.ptr, _stream(stream)))
+    ws.check(stream)
+    return D
 
 
 def attention_fwd_sage(ops: dict, N: int, softmax_scale: float | None = None, O=None, lse=None,

@@ -241,6 +241,43 @@ int vca_attention_fwd(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq
                       const vca_bf16* v_mean, int B, int H, int N, int d, float softmax_scale,
                       vca_bf16* O, float* lse, void* ws, size_t ws_bytes, vca_stream_t stream);
 
+/* Attention of the 4-bit V-Smooth variant ([VCA-mtp] abstract: 4-bit V-Smooth;
+ * ExpCast is 8-bit only, so the probabilities are exponentials quantised to
+ * NVFP4; [TRT-blog] formats table: NVFP4 = E2M1 elements, one E4M3 scale per 16
+ * elements, one fp32 scale per tensor).  Inputs are the outputs of
+ * vca_smooth_quantize_qkv_fp4 (Qq, q_scale, Kq, k_scale as the 8-bit prep; VrT4
+ * [B][H][d][Np/2] E2M1 codes, low nibble = even token; v_sc [B][H][d][Np/16]
+ * E4M3 group scales, 8-byte aligned; v_gscale [B][H] fp32 head scales G).
+ * z, the reference n and its rescale rule are those of vca_attention_fwd; then
+ * for each row and key block, per 16 keys g:
+ *   p_j  = 2^(z_ij - n - phi + 4) in fp32
+ *   sc_g = e4m3(max_{j in g} p_j / 0.75), s_g = 2^-3 decode(sc_g)
+ *   p^_j = s_g e2m1(p_j * (1 / s_g))       (one fp32 rounding per step)
+ *   l_ib = sum of p^_j over key block b
+ *   O_i  = (sum_j p^_j G s_v e2m1(VrT4) + sum_b l_ib v_mean[b]) / sum_b l_ib
+ *   lse_i = ln 2 * (n + phi - 4 + log2 sum_b l_ib)   (optional)
+ * PV runs as tcgen05 kind::mxf4nvf4 block-scaled MMAs.  Errors as
+ * vca_attention_fwd; VCA_ERR_INVALID if v_sc is not 8-byte aligned. */
+int vca_attention_fwd_fp4(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                          const float* k_scale, const uint8_t* VrT4, const uint8_t* v_sc,
+                          const float* v_gscale, const vca_bf16* v_mean, int B, int H, int N, int d,
+                          float softmax_scale, vca_bf16* O, float* lse, void* ws, size_t ws_bytes,
+                          vca_stream_t stream);
+
+/* Check of the block-scaled FP4 MMA that vca_attention_fwd_fp4 runs: one
+ * 128x128x128 product in one CTA with known operands.  The pages have no
+ * counterpart (a library self-test of the operand and scale-factor layouts).
+ * All device pointers, 16-byte aligned:
+ *   a_codes [128][64] bytes   A rows, E2M1 codes, low nibble = even column
+ *   sf_cols [128][64] bytes   tensor-memory lane l, columns 0..15 (4 bytes
+ *                             each): the A scale factors of K step k (64
+ *                             columns of A) from column 4k, B's from 8 + 4k
+ *   b_codes [128][64] bytes   B^T rows (one per output column), as a_codes
+ *   D       [128][128] fp32   out: the product with the scales applied
+ *   ws      status word (a wait that runs out records VCA_ERR_TIMEOUT) */
+int vca_debug_fp4_mma(const uint8_t* a_codes, const uint8_t* sf_cols, const uint8_t* b_codes, float* D,
+                      void* ws, vca_stream_t stream);
+
 /* Same attention with Skip Softmax (BLASST) block rejection ([TRT-blog],
  * section "Sparse Attention with Skip Softmax": a score block is dropped for a
  * query row when exp(block max - running max) < lambda; dropped blocks skip the
