@@ -219,7 +219,18 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     ws4.check()
     fp4_ms = f0.elapsed_time(f1) / reps
-    del ops4
+    # ---- attention of the 4-bit variant (NVFP4 P and V residual in PV) on those operands
+    O4 = vca.attention_fwd_fp4(ops4, N, scale, ws=ws4)
+    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a0.record(stream)
+    for _ in range(3):
+        vca.attention_fwd_fp4(ops4, N, scale, O=O4, ws=ws4)
+    a1.record(stream)
+    torch.cuda.synchronize()
+    ws4.check()
+    fp4_attn_ms = a0.elapsed_time(a1) / 3
+    del ops4, O4
 
     # ---- in-repo BF16 comparator on the same shapes
     bf16_ms = None
@@ -420,6 +431,9 @@ def run_ours(args, world, rank, local):
                         "frac": round(fb / (fp4_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                         "launches": 4, "what": "vca_smooth_quantize_qkv_fp4: Q/K E4M3 as the 8-bit prep, "
                                               "V residual NVFP4 (two passes over V)"}
+    line["fp4_attention"] = {"ms": round(fp4_attn_ms, 3), "tflops": round(w.flops / (fp4_attn_ms / 1e3) / 1e12, 1),
+                             "what": "vca_attention_fwd_fp4: QK^T E4M3, PV kind::mxf4nvf4 with NVFP4 probabilities "
+                                     "(exp2 on the MUFU pipe) and NVFP4 V residual"}
     pb = prep_algorithmic_bytes(w)
     line["prep_roofline"] = {"bound": "hbm", "algorithmic_bytes": pb,
                              "achieved": round(pb / (prep_ms / 1e3) / 1e9, 1), "unit": "GB/s",
