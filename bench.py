@@ -155,8 +155,8 @@ def run_ours(args, world, rank, local):
     ops = vca.alloc_quantized(B, H, N, dev)
     O = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
-    # init, T x (assign, sort count, sort scan, sort scatter, accumulate, update), quantise x2, attention
-    launches_per_step = 1 + 6 * KMEANS_ITERS + 2 + 1
+    # init, T x (assign, sort count, sort scan, sort scatter, accumulate, update), quantise, attention
+    launches_per_step = 1 + 6 * KMEANS_ITERS + 1 + 1
 
     def step(t_attn=None):
         _, _, perm = vca.cluster_permute(V, w.k, KMEANS_ITERS, ws=ws)

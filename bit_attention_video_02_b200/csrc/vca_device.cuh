@@ -300,15 +300,18 @@ __device__ __forceinline__ uint16_t double_to_bf16_rne(double x) {
 }
 
 // Exact split of llrint(v * 2^24) for |v| < 2^20 (at most 45 bits) into
-// hi * 2^22 + lo with |hi|, |lo| < 2^22, using float operations only: f = v * 2^24
-// is exact, hi = trunc(f / 2^22), lo = rne(f - hi * 2^22) (the only rounding, the
-// same as llrint's); each becomes an integer through the magic-number add.
+// hi * 2^22 + lo with |hi| < 2^22, |lo| <= 2^21, using float operations only:
+// f = v * 2^24 is exact, hi = rne(f / 2^22) by the magic-number add (f / 2^22
+// is exact), lo = rne(f - hi * 2^22) (the remainder is exact; its rounding is
+// the only one, the same as llrint's since hi * 2^22 is an integer); each
+// becomes an integer through the magic-number add.  No conversion instruction.
 __device__ __forceinline__ void fix24_split(float v, int& hi, int& lo) {
   const float kMagic = 12582912.0f;   // 1.5 * 2^23
   const float f = v * 16777216.0f;
-  const float hf = truncf(f * 2.384185791015625e-07f);     // f / 2^22, truncated
-  const float lf = __fmaf_rn(hf, -4194304.0f, f);         // exact remainder
-  hi = (int)(__float_as_uint(hf + kMagic) - 0x4B400000u);
+  const float hm = __fadd_rn(f * 2.384185791015625e-07f, kMagic);   // 1.5 * 2^23 + rne(f / 2^22)
+  const float hf = __fsub_rn(hm, kMagic);
+  const float lf = __fmaf_rn(hf, -4194304.0f, f);                   // exact remainder
+  hi = (int)(__float_as_uint(hm) - 0x4B400000u);
   lo = (int)(__float_as_uint(lf + kMagic) - 0x4B400000u);
 }
 

@@ -1,4 +1,4 @@
-// vca_prep.cu -- V-Smooth quantisation of Q, K and V (one fused launch).
+// vca_prep.cu -- V-Smooth quantisation of Q, K and V.
 //
 // Method: "VC-Attention: Training-Free Low-Bit Attention Speeds Video Diffusion
 // Up to 3.6x" (V-Smooth bullet): value tokens are reordered so each hardware
@@ -7,12 +7,18 @@
 // mean is stored exactly; "Nunchux AI Introduces VC-Attention..." (abstract):
 // a mean costs 0.125 bit per value element (16 bits per 128 tokens).
 //
-// One CTA per (128-token block, tensor, head): 256 threads, HBM-bound; Q/K and
-// V blocks are two launches of the same kernel (only V uses shared memory).  Loads
-// are 16-byte vectors of whole token rows (gathered through the permutation for
-// K and V); Q/K codes are written straight from registers, the V residual is
-// transposed through shared memory so VrT rows (channel-major) are written as
-// full 128-byte lines.
+// vca_smooth_quantize_qkv runs one persistent kernel (smooth_quant_stream_kernel):
+// a producer warp streams 128-token tiles of Q, K and V (K and V rows gathered
+// through the permutation) into a 3-stage shared-memory ring with bulk
+// asynchronous copies, and 8 compute warps code one tile while two more land.
+// Q/K tiles: per-block fp32 scale, codes written straight from registers.
+// V tiles: each thread holds 8 consecutive tokens x 8 channels; exact
+// per-channel sums and the residual maximum through shared-memory reductions;
+// the residual codes are transposed in registers so VrT rows (channel-major)
+// are written as full 128-byte lines.  smooth_quant_kernel (one CTA per Q or K
+// block) serves the 4-bit prep's Q and K.
+#include <algorithm>
+
 #include "vca_device.cuh"
 #include "vca_host.h"
 
@@ -69,13 +75,10 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return m;
 }
 
+// The Q and K blocks: one CTA per (128-token block, tensor, head), tensor =
+// blockIdx.y + tensor_base (0 = Q, 1 = K).
 __global__ void __launch_bounds__(kPrepThreads) smooth_quant_kernel(const PrepArgs a) {
-  extern __shared__ __align__(16) uint8_t sm[];
-  uint16_t* tile = reinterpret_cast<uint16_t*>(sm);                         // [128][136] bf16
-  uint8_t* codeT = sm + 128 * kTilePitch * 2;                               // [128][144] u8
   __shared__ float red[kPrepThreads / 32];
-  __shared__ long long psum[kPrepThreads];
-  __shared__ float mu_s[128];
   __shared__ int flag_s;
 
   const int blk = blockIdx.x, tensor = blockIdx.y + a.tensor_base, bh = blockIdx.z;
@@ -87,7 +90,7 @@ __global__ void __launch_bounds__(kPrepThreads) smooth_quant_kernel(const PrepAr
   const int chunk = t & 15;          // 16-byte chunk (8 channels) of a row
   const int rsub = t >> 4;           // 0..15
 
-  const uint16_t* src = tensor == 0 ? a.Q : (tensor == 1 ? a.K : a.V);
+  const uint16_t* src = tensor == 0 ? a.Q : a.K;
   src += (int64_t)bh * N * 128;
   const int32_t* perm = a.perm + (int64_t)bh * N;
   if (t == 0) flag_s = 0;
@@ -111,13 +114,12 @@ __global__ void __launch_bounds__(kPrepThreads) smooth_quant_kernel(const PrepAr
         amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
         uint32_t elo = (ws4[q] >> 7) & 0xFFu, ehi = (ws4[q] >> 23) & 0xFFu;
         bad |= (elo == 0xFF) | (ehi == 0xFF);
-        if (tensor == 2) bad |= (elo >= 147) | (ehi >= 147);   // |v| >= 2^20
       }
     }
   }
   if (bad) flag_s = 1;
 
-  if (tensor < 2) {
+  {
     // ---- Q / K: per-block fp32 scale, codes straight from registers
     float m = block_max(amax, red);
     if (flag_s && t == 0) report(a.st, VCA_ERR_NONFINITE, 1 + tensor, blk);
@@ -145,76 +147,304 @@ __global__ void __launch_bounds__(kPrepThreads) smooth_quant_kernel(const PrepAr
     return;
   }
 
-  // ---- V: stage the block in shared memory
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    int row = it * 16 + rsub;
-    *reinterpret_cast<uint4*>(tile + row * kTilePitch + chunk * 8) = w[it];
-  }
-  __syncthreads();
-  if (flag_s && t == 0) report(a.st, VCA_ERR_NONFINITE, 3, blk);
+}
 
-  // exact per-channel sums in 2^-24 fixed point: two threads per channel
-  const int ch = t & 127, half = t >> 7;
-  long long s = 0;
-  for (int r = half * 64; r < min(nv, half * 64 + 64); ++r) {
-    float v = __uint_as_float((uint32_t)tile[r * kTilePitch + ch] << 16);
-    s += __float2ll_rn(v * 16777216.0f);
-  }
-  psum[t] = s;
-  __syncthreads();
-  if (t < 128) {
-    long long S = psum[t] + psum[t + 128];
-    double mean = __ddiv_rn((double)S, (double)nv * 16777216.0);
-    uint16_t mb = double_to_bf16_rne(mean);
-    a.v_mean[((int64_t)bh * nb + blk) * 128 + t] = mb;
-    mu_s[t] = __uint_as_float((uint32_t)mb << 16);
-  }
-  __syncthreads();
 
-  // residual max over the valid tokens and all channels
-  float mu = mu_s[ch];
-  float ramax = 0.0f;
-  for (int r = half * 64; r < min(nv, half * 64 + 64); ++r) {
-    float v = __uint_as_float((uint32_t)tile[r * kTilePitch + ch] << 16);
-    ramax = fmaxf(ramax, fabsf(__fsub_rn(v, mu)));
-  }
-  float m = block_max(ramax, red);
-  int e = v_exponent(m);
-  if (t == 0) a.v_exp[(int64_t)bh * nb + blk] = (int8_t)e;
-  float sc = pow2_neg(e);
 
-  // codes for (channel, 16 tokens) units -> transposed code tile
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    int t0 = (half + 2 * i) * 16;
-    uint32_t pk[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float x[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        int r = t0 + q * 4 + u;
-        float v = __uint_as_float((uint32_t)tile[r * kTilePitch + ch] << 16);
-        x[u] = r < nv ? __fmul_rn(__fsub_rn(v, mu), sc) : 0.0f;
-      }
-      pk[q] = (uint32_t)cvt_e4m3x2(x[0], x[1]) | ((uint32_t)cvt_e4m3x2(x[2], x[3]) << 16);
+// 4 x 4 byte transpose: out[c] byte r = in[r] byte c.
+__device__ __forceinline__ void transpose4x4(const uint32_t in[4], uint32_t out[4]) {
+  const uint32_t t0 = prmt(in[0], in[1], 0x5140u), t1 = prmt(in[0], in[1], 0x7362u);
+  const uint32_t t2 = prmt(in[2], in[3], 0x5140u), t3 = prmt(in[2], in[3], 0x7362u);
+  out[0] = prmt(t0, t2, 0x5410u);
+  out[1] = prmt(t0, t2, 0x7632u);
+  out[2] = prmt(t1, t3, 0x5410u);
+  out[3] = prmt(t1, t3, 0x7632u);
+}
+
+
+// ---------------------------------------------------------------- streaming form
+// vca_smooth_quantize_qkv's kernel: persistent CTAs walk the (block, tensor,
+// head) items; a producer warp (warp 8) fills a 3-stage ring of 32 KB token
+// tiles with bulk asynchronous copies (one copy for a block of Q, whose rows
+// are contiguous; one 256-byte copy per gathered row of K or V), so two blocks
+// stream in while the 8 compute warps code one.  The compute warps synchronise
+// among themselves on named barrier 1 and release a stage with one arrival
+// per warp.  The arithmetic per block is that of smooth_quant_kernel for Q
+// and K; the V scratch (exact partial sums and the
+// code tile) reuses the stage of the block being coded.
+constexpr int kStreamStages = 3;
+constexpr uint32_t kStageBytes = 128 * 256;
+constexpr size_t kStreamSmem = kStreamStages * kStageBytes + 128;
+constexpr int kStreamThreads = kPrepThreads + 32;
+
+__device__ __forceinline__ void compute_sync() {   // the 256 compute threads
+  asm volatile("bar.sync 1, %0;" ::"n"(kPrepThreads) : "memory");
+}
+__device__ __forceinline__ int compute_sync_or(int pred) {
+  int r;
+  asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\tbar.red.or.pred q, 1, %2, p;\n\t"
+               "selp.s32 %0, 1, 0, q;\n\t}"
+               : "=r"(r)
+               : "r"(pred), "n"(kPrepThreads)
+               : "memory");
+  return r;
+}
+__device__ __forceinline__ float compute_max(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  compute_sync();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  compute_sync();
+  float m = red[0];
+  for (int i = 1; i < kPrepThreads / 32; ++i) m = fmaxf(m, red[i]);
+  return m;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Per 16-bit half, the larger of the two bf16 magnitude bit patterns (for
+// finite values these order like the magnitudes; inf and NaN are larger).
+__device__ __forceinline__ uint32_t vmax_mag2(uint32_t acc, uint32_t w) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w & 0x7FFF7FFFu));
+  return r;
+}
+__device__ __forceinline__ uint32_t max_half(uint32_t m2) { return max(m2 & 0xFFFFu, m2 >> 16); }
+
+__global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(const PrepArgs a, int BH,
+                                                                                 unsigned long long lim) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ uint64_t full[kStreamStages];
+  __shared__ uint64_t empty[kStreamStages];
+  __shared__ float red[kPrepThreads / 32];
+  __shared__ float mu_s[128];
+  __shared__ int abort_s;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int N = a.N, nb = a.nb;
+  const int64_t Np = (int64_t)nb * 128;
+  const long long items = 3ll * BH * nb;
+  if (t == 0) {
+    abort_s = 0;
+    for (int i = 0; i < kStreamStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kPrepThreads / 32);
     }
-    *reinterpret_cast<uint4*>(codeT + ch * kCodePitch + t0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    fence_barrier_init();
   }
   __syncthreads();
-  // coalesced write: each VrT row (one channel) gets 128 bytes at tokens n0..n0+127
-  uint8_t* dstT = a.VrT + (int64_t)bh * 128 * Np + n0;
+  // item -> (tensor, head, block): tensors interleaved so a CTA mixes all three
+  auto decode = [&](long long it, int& tensor, int& bh, int& blk) {
+    tensor = (int)(it % 3);
+    const long long rest = it / 3;
+    bh = (int)(rest / nb);
+    blk = (int)(rest % nb);
+  };
+  const long long first = blockIdx.x, step = gridDim.x;
+  if (warp == kPrepThreads / 32) {
+    // ---- producer: item k goes to stage k % 3 once the compute warps released it
+    int k = 0;
+    for (long long it = first; it < items; it += step, ++k) {
+      const int stg = k % kStreamStages;
+      if (k >= kStreamStages &&
+          !mbar_wait_bounded(&empty[stg], ((k / kStreamStages) - 1) & 1, &abort_s, a.st, lim, 803))
+        break;
+      int tensor, bh, blk;
+      decode(it, tensor, bh, blk);
+      const int n0 = blk * 128, nv = min(128, N - n0);
+      uint8_t* dst = stages + stg * kStageBytes;
+      // the gathered rows' source indices first (one round trip), then the copies
+      int src_row[4];
+      if (tensor != 0) {
+        const int32_t* pm = a.perm + (int64_t)bh * N + n0;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    int idx = i * kPrepThreads + t;       // 0..1023
-    int c = idx >> 3, part = idx & 7;
-    *reinterpret_cast<uint4*>(dstT + (int64_t)c * Np + part * 16) =
-        *reinterpret_cast<const uint4*>(codeT + c * kCodePitch + part * 16);
+        for (int i = 0; i < 4; ++i) src_row[i] = lane + 32 * i < nv ? __ldg(pm + lane + 32 * i) : 0;
+      }
+      if (lane == 0) mbar_arrive_expect_tx(&full[stg], (uint32_t)nv * 256u);
+      __syncwarp();
+      if (tensor == 0) {
+        if (lane == 0) bulk_g2s(dst, a.Q + ((int64_t)bh * N + n0) * 128, (uint32_t)nv * 256u, &full[stg]);
+      } else {
+        const uint16_t* src = (tensor == 1 ? a.K : a.V) + (int64_t)bh * N * 128;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = lane + 32 * i;
+          if (r < nv) bulk_g2s(dst + r * 256, src + (int64_t)src_row[i] * 128, 256u, &full[stg]);
+        }
+      }
+    }
+    return;
+  }
+  int k = 0;
+  for (long long it = first; it < items; it += step, ++k) {
+    const int stg = k % kStreamStages;
+    uint8_t* tile = stages + stg * kStageBytes;
+    bool ok = mbar_wait_bounded(&full[stg], (k / kStreamStages) & 1, &abort_s, a.st, lim, 800);
+    if (compute_sync_or(!ok)) break;
+    int tensor, bh, blk;
+    decode(it, tensor, bh, blk);
+    const int n0 = blk * 128, nv = min(128, N - n0);
+    if (tensor < 2) {
+      // ---- Q / K: per-block fp32 scale, codes straight from registers
+      const int chunk = t & 15, rsub = t >> 4;
+      uint4 w[8];
+      uint32_t m2 = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = i * 16 + rsub;
+        w[i] = row < nv ? *reinterpret_cast<const uint4*>(tile + row * 256 + chunk * 16) : make_uint4(0, 0, 0, 0);
+        m2 = vmax_mag2(vmax_mag2(m2, w[i].x), w[i].y);
+        m2 = vmax_mag2(vmax_mag2(m2, w[i].z), w[i].w);
+      }
+      const uint32_t mbits = max_half(m2);
+      const float m = compute_max(__uint_as_float(mbits << 16), red);   // block max |x| (inf / NaN flagged)
+      if (compute_sync_or(mbits >= 0x7F80u) && t == 0) report(a.st, VCA_ERR_NONFINITE, 1 + tensor, blk);
+      const float inv = m > 0.0f ? __fdiv_rn(448.0f, m) : 0.0f;
+      if (t == 0) (tensor == 0 ? a.q_scale : a.k_scale)[(int64_t)bh * nb + blk] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+      uint8_t* dst = (tensor == 0 ? a.Qq : a.Kq) + ((int64_t)bh * Np + n0) * 128;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int row = i * 16 + rsub;
+        const uint32_t ws4[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+        uint32_t c[2] = {0u, 0u};
+        if (row < nv && m > 0.0f) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            c[q >> 1] |= (uint32_t)cvt_e4m3x2(__fmul_rn(bf16_lo(ws4[q]), inv), __fmul_rn(bf16_hi(ws4[q]), inv))
+                         << ((q & 1) * 16);
+        }
+        *reinterpret_cast<uint2*>(dst + (int64_t)row * 128 + chunk * 8) = make_uint2(c[0], c[1]);
+      }
+    } else {
+      // ---- V: thread = 8 consecutive tokens x 8 channels
+      const int chunk = t & 15, g = t >> 4;
+      uint4 w[8];
+      uint32_t m2 = 0u;
+      int hs[8], ls[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) hs[c] = ls[c] = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int row = 8 * g + u;
+        w[u] = row < nv ? *reinterpret_cast<const uint4*>(tile + row * 256 + chunk * 16) : make_uint4(0, 0, 0, 0);
+        m2 = vmax_mag2(vmax_mag2(m2, w[u].x), w[u].y);
+        m2 = vmax_mag2(vmax_mag2(m2, w[u].z), w[u].w);
+        const uint32_t ws4[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          int h, l;
+          fix24_split(bf16_lo(ws4[q]), h, l);
+          hs[2 * q] += h;
+          ls[2 * q] += l;
+          fix24_split(bf16_hi(ws4[q]), h, l);
+          hs[2 * q + 1] += h;
+          ls[2 * q + 1] += l;
+        }
+      }
+      // the tile is in registers: its stage now holds the partial sums and codes
+      const bool anybad = compute_sync_or(max_half(m2) >= 0x4980u);   // |v| >= 2^20, inf or NaN
+      if (anybad && t == 0) report(a.st, VCA_ERR_NONFINITE, 3, blk);
+      int* s_hi = reinterpret_cast<int*>(tile);
+      int* s_lo = s_hi + 16 * 128;
+      uint8_t* codeT = tile + 2 * 16 * 128 * 4;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        s_hi[g * 128 + 8 * chunk + c] = hs[c];
+        s_lo[g * 128 + 8 * chunk + c] = ls[c];
+      }
+      compute_sync();
+      if (t < 128) {
+        int H = 0, L = 0;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          H += s_hi[q * 128 + t];
+          L += s_lo[q * 128 + t];
+        }
+        const long long S = (long long)H * 4194304ll + (long long)L;
+        const uint16_t mb = double_to_bf16_rne(__ddiv_rn((double)S, (double)nv * 16777216.0));
+        a.v_mean[((int64_t)bh * nb + blk) * 128 + t] = mb;
+        mu_s[t] = __uint_as_float((uint32_t)mb << 16);
+      }
+      compute_sync();
+      float mu[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mu[c] = mu_s[8 * chunk + c];
+      float ramax = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (8 * g + u < nv) {
+          const uint32_t ws4[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            ramax = fmaxf(ramax, fabsf(__fsub_rn(bf16_lo(ws4[q]), mu[2 * q])));
+            ramax = fmaxf(ramax, fabsf(__fsub_rn(bf16_hi(ws4[q]), mu[2 * q + 1])));
+          }
+        }
+      }
+      const float m = compute_max(ramax, red);
+      const int e = v_exponent(m);
+      if (t == 0) a.v_exp[(int64_t)bh * nb + blk] = (int8_t)e;
+      const float sc = pow2_neg(e);
+      uint32_t lo4[8], hi4[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t ws4[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+        float x[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          x[2 * q] = __fmul_rn(__fsub_rn(bf16_lo(ws4[q]), mu[2 * q]), sc);
+          x[2 * q + 1] = __fmul_rn(__fsub_rn(bf16_hi(ws4[q]), mu[2 * q + 1]), sc);
+        }
+        const bool valid = 8 * g + u < nv;
+        lo4[u] = valid ? ((uint32_t)cvt_e4m3x2(x[0], x[1]) | ((uint32_t)cvt_e4m3x2(x[2], x[3]) << 16)) : 0u;
+        hi4[u] = valid ? ((uint32_t)cvt_e4m3x2(x[4], x[5]) | ((uint32_t)cvt_e4m3x2(x[6], x[7]) << 16)) : 0u;
+      }
+      uint32_t cT[8][2];
+      {
+        uint32_t o[4];
+        transpose4x4(lo4, o);
+        for (int c = 0; c < 4; ++c) cT[c][0] = o[c];
+        transpose4x4(lo4 + 4, o);
+        for (int c = 0; c < 4; ++c) cT[c][1] = o[c];
+        transpose4x4(hi4, o);
+        for (int c = 0; c < 4; ++c) cT[4 + c][0] = o[c];
+        transpose4x4(hi4 + 4, o);
+        for (int c = 0; c < 4; ++c) cT[4 + c][1] = o[c];
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int c = 8 * chunk + i;
+        *reinterpret_cast<uint2*>(codeT + c * 128 + 8 * (g ^ vseg_swz(c))) = make_uint2(cT[i][0], cT[i][1]);
+      }
+      compute_sync();
+      uint8_t* dstT = a.VrT + (int64_t)bh * 128 * Np + n0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int idx = i * kPrepThreads + t;
+        const int c = idx >> 3, part = idx & 7;
+        *reinterpret_cast<uint4*>(dstT + (int64_t)c * Np + 16 * (part ^ (vseg_swz(c) >> 1))) =
+            *reinterpret_cast<const uint4*>(codeT + c * 128 + part * 16);
+      }
+    }
+    // this warp is done with the stage (its reads and, for V, the scratch)
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stg]);
+  }
+  if (abort_s) {
+    // let copies already issued land before the CTA exits
+    for (int i = 0; i < kStreamStages; ++i) {
+      int never = 0;
+      mbar_wait_bounded(&full[i], 0, &never, nullptr, lim, 801);
+      mbar_wait_bounded(&full[i], 1, &never, nullptr, lim, 802);
+    }
   }
 }
 
-constexpr size_t kPrepSmem = 128 * kTilePitch * 2 + 128 * kCodePitch;
+
 
 // ---------------------------------------------------------------- 4-bit V-Smooth
 // "Nunchux AI Introduces VC-Attention..." (abstract): a 4-bit V-Smooth serves
@@ -404,22 +634,20 @@ extern "C" int vca_smooth_quantize_qkv(const vca_bf16* Q, const vca_bf16* K, con
     if (!aligned16(p)) return fail(VCA_ERR_INVALID, "vca_smooth_quantize_qkv: tensors must be 16-byte aligned");
   if (!ws || ws_bytes < vca_smooth_quantize_workspace_size(B, H, N))
     return fail(VCA_ERR_WORKSPACE, "vca_smooth_quantize_qkv: workspace too small");
-  if (cudaFuncSetAttribute(smooth_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kPrepSmem) != cudaSuccess)
+  if (cudaFuncSetAttribute(smooth_quant_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kStreamSmem) != cudaSuccess)
     return fail(VCA_ERR_CUDA, "vca_smooth_quantize_qkv: cannot set shared-memory size");
   PrepArgs a;
   a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.N = N; a.nb = (N + 127) / 128;
   a.Qq = Qq; a.q_scale = q_scale; a.Kq = Kq; a.k_scale = k_scale; a.VrT = VrT;
   a.v_exp = v_exp; a.v_mean = v_mean; a.st = (DevStatus*)ws;
-  // Q and K blocks need no shared tile: a launch of their own keeps them at full
-  // occupancy; the V blocks (mean, residual, transpose) get the shared tile
   a.tensor_base = 0;
-  smooth_quant_kernel<<<dim3(a.nb, 2, B * H), kPrepThreads, 0, (cudaStream_t)stream>>>(a);
-  int rc = check_launch("smooth_quant_kernel (Q, K)");
-  if (rc) return rc;
-  a.tensor_base = 2;
-  smooth_quant_kernel<<<dim3(a.nb, 1, B * H), kPrepThreads, kPrepSmem, (cudaStream_t)stream>>>(a);
-  return check_launch("smooth_quant_kernel (V)");
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long items = 3ll * B * H * a.nb;
+  const int grid = (int)std::min<long long>(items, 2ll * sms);   // two resident CTAs per SM
+  smooth_quant_stream_kernel<<<grid, kStreamThreads, kStreamSmem, (cudaStream_t)stream>>>(a, B * H, wait_limit_ns());
+  return check_launch("smooth_quant_stream_kernel");
 }
 
 extern "C" size_t vca_smooth_quantize_fp4_workspace_size(int B, int H, int N) {
