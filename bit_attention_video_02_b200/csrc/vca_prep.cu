@@ -162,6 +162,12 @@ __device__ __forceinline__ void transpose4x4(const uint32_t in[4], uint32_t out[
 }
 
 
+// V code tile: 128 channel rows of 128 bytes; the 8-byte segment of tokens
+// 8 g .. 8 g + 7 of channel c sits at segment g ^ (2 ((c >> 3) & 7)), so the 32
+// threads of a warp storing one channel each hit 16 bank pairs twice, and
+// 16-byte parts keep adjacent token segments together.
+__device__ __forceinline__ int vseg_swz(int c) { return 2 * ((c >> 3) & 7); }
+
 // ---------------------------------------------------------------- streaming form
 // vca_smooth_quantize_qkv's kernel: persistent CTAs walk the (block, tensor,
 // head) items; a producer warp (warp 8) fills a 3-stage ring of 32 KB token
