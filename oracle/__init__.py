@@ -78,6 +78,8 @@ def _declare(L):
     L.vo_smooth_quantize_head_vhead.argtypes = [vp] * 4 + [i32, i32] + [vp] * 7
     L.vo_sage_quantize_head.argtypes = [vp] * 3 + [i32, i32] + [vp] * 7
     L.vo_attention_head_sage.argtypes = [vp] * 6 + [i32, i32, f64, vp, i32, i32, vp, vp]
+    L.vo_sage_quantize_head_i8.argtypes = [vp] * 3 + [i32, i32] + [vp] * 7
+    L.vo_attention_head_sage_i8.argtypes = [vp] * 6 + [i32, i32, f64, vp, i32, i32, vp, vp]
     L.vo_attention_head_skip.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, f64, vp, vp, vp]
     L.vo_attention_head_ex.argtypes = [vp] * 7 + [i32, i32, f64, vp, i32, i32, f64, vp, vp, vp, vp, vp]
     L.vo_attention_head_bf16_skip.argtypes = [vp] * 4 + [i32, i32, f64, vp, i32, i32, f64, vp]
@@ -236,20 +238,24 @@ def smooth_quantize_head_fp4(Q, K, V, perm):
     return out
 
 
-def sage_quantize_head(Q, K, V):
+def sage_quantize_head(Q, K, V, qk_dtype: str = "fp8"):
     """One head of the SAGE-style comparison quantisation (per-token Q,
-    per-16-token K after K-mean smoothing, per-channel V; no reordering)."""
+    per-16-token K after K-mean smoothing, per-channel V; no reordering).
+    qk_dtype "fp8" codes Q and K' as E4M3 (uint8), "int8" as signed bytes."""
+    if qk_dtype not in ("fp8", "int8"):
+        raise ValueError(f"qk_dtype must be 'fp8' or 'int8', not {qk_dtype!r}")
     Q, K, V = (np.ascontiguousarray(a, dtype=np.uint16) for a in (Q, K, V))
     N, d = Q.shape
     Np = (N + BLOCK - 1) // BLOCK * BLOCK
+    ct = np.int8 if qk_dtype == "int8" else np.uint8
     out = dict(
-        Qq=np.zeros((Np, d), np.uint8), q_scale=np.empty(Np, np.float32),
-        Kq=np.zeros((Np, d), np.uint8), k_scale=np.empty(Np // 16, np.float32),
+        Qq=np.zeros((Np, d), ct), q_scale=np.empty(Np, np.float32),
+        Kq=np.zeros((Np, d), ct), k_scale=np.empty(Np // 16, np.float32),
         VcT=np.zeros((d, Np), np.uint8), v_chscale=np.empty(d, np.float32),
         k_mean=np.empty(d, np.uint16))
-    lib().vo_sage_quantize_head(
-        _p(Q), _p(K), _p(V), N, d, _p(out["Qq"]), _p(out["q_scale"]), _p(out["Kq"]), _p(out["k_scale"]),
-        _p(out["VcT"]), _p(out["v_chscale"]), _p(out["k_mean"]))
+    fn = lib().vo_sage_quantize_head_i8 if qk_dtype == "int8" else lib().vo_sage_quantize_head
+    fn(_p(Q), _p(K), _p(V), N, d, _p(out["Qq"]), _p(out["q_scale"]), _p(out["Kq"]), _p(out["k_scale"]),
+       _p(out["VcT"]), _p(out["v_chscale"]), _p(out["k_mean"]))
     return out
 
 
@@ -312,16 +318,19 @@ def attention_head_bf16(Q, K, V, perm, softmax_scale: float, rows=None, flags: i
 
 
 def attention_head_sage(ops: dict, N: int, softmax_scale: float, rows=None, flags: int = 0):
-    """Attention on SAGE-style operands (dict from ``sage_quantize_head``).
+    """Attention on SAGE-style operands (dict from ``sage_quantize_head``; the
+    Q/K code dtype, uint8 E4M3 or int8, picks the decoding).
     Returns (O [nrows, d] fp64, lse [nrows])."""
     rows = _rows(rows, N)
     d = ops["Qq"].shape[1]
     O = np.empty((rows.shape[0], d), np.float64)
     lse = np.empty(rows.shape[0], np.float64)
     c = {k: np.ascontiguousarray(v) for k, v in ops.items()}
-    lib().vo_attention_head_sage(
-        _p(c["Qq"]), _p(c["q_scale"]), _p(c["Kq"]), _p(c["k_scale"]), _p(c["VcT"]), _p(c["v_chscale"]),
-        N, d, float(softmax_scale), _p(rows), rows.shape[0], int(flags), _p(O), _p(lse))
+    if c["Qq"].dtype != c["Kq"].dtype or c["Qq"].dtype not in (np.uint8, np.int8):
+        raise ValueError("Qq and Kq must both be uint8 (E4M3) or both int8")
+    fn = lib().vo_attention_head_sage_i8 if c["Qq"].dtype == np.int8 else lib().vo_attention_head_sage
+    fn(_p(c["Qq"]), _p(c["q_scale"]), _p(c["Kq"]), _p(c["k_scale"]), _p(c["VcT"]), _p(c["v_chscale"]),
+       N, d, float(softmax_scale), _p(rows), rows.shape[0], int(flags), _p(O), _p(lse))
     return O, lse
 
 

@@ -526,9 +526,34 @@ static void quant_group(const float* x, int n, uint8_t* out, float* scale) {
     for (int i = 0; i < n; ++i) out[i] = vo_e4m3_encode(x[i] * inv);
 }
 
-void vo_sage_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int N, int d,
-                           uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
-                           uint8_t* VcT, float* v_chscale, uint16_t* k_mean) {
+/* The INT8 form of the same per-group rule, the post's other qk_dtype (int8,
+ * the one it uses): scale = amax / 127, code = rne(x * (127 / amax)) with the
+ * product in fp32, a signed byte in [-127, 127]; an all-zero group has scale 1
+ * and codes 0. */
+static void quant_group_i8(const float* x, int n, int8_t* out, float* scale) {
+    float amax = 0.0f;
+    for (int i = 0; i < n; ++i)
+        if (fabsf(x[i]) > amax) amax = fabsf(x[i]);
+    if (!(amax > 0.0f)) {
+        *scale = 1.0f;
+        memset(out, 0, (size_t)n);
+        return;
+    }
+    *scale = amax / 127.0f;
+    float inv = 127.0f / amax;
+    for (int i = 0; i < n; ++i) {
+        float r = nearbyintf(x[i] * inv);   /* round half to even (default mode) */
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        out[i] = (int8_t)r;
+    }
+}
+
+/* Q and K' groups coded as E4M3 (qk_i8 = 0, Qq/Kq uint8) or INT8 (qk_i8 = 1,
+ * Qq/Kq int8); V, k_mean and the layouts are the same in both. */
+static void sage_quantize(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int N, int d, void* Qq,
+                          float* q_scale, void* Kq, float* k_scale, uint8_t* VcT, float* v_chscale,
+                          uint16_t* k_mean, int qk_i8) {
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
     int64_t Np = (int64_t)nb * VO_BLOCK;
     memset(Qq, 0, (size_t)Np * d);
@@ -544,14 +569,20 @@ void vo_sage_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_t*
     }
     for (int j = 0; j < N; ++j) {
         for (int c = 0; c < d; ++c) x[c] = vo_bf16_to_float(Q[(int64_t)j * d + c]);
-        quant_group(x, d, Qq + (int64_t)j * d, &q_scale[j]);
+        if (qk_i8)
+            quant_group_i8(x, d, (int8_t*)Qq + (int64_t)j * d, &q_scale[j]);
+        else
+            quant_group(x, d, (uint8_t*)Qq + (int64_t)j * d, &q_scale[j]);
     }
     for (int g = 0; g * 16 < N; ++g) {
         int n = N - g * 16 < 16 ? N - g * 16 : 16;
         for (int t = 0; t < n; ++t)
             for (int c = 0; c < d; ++c)
                 x[t * d + c] = vo_bf16_to_float(K[(int64_t)(g * 16 + t) * d + c]) - vo_bf16_to_float(k_mean[c]);
-        quant_group(x, n * d, Kq + (int64_t)g * 16 * d, &k_scale[g]);
+        if (qk_i8)
+            quant_group_i8(x, n * d, (int8_t*)Kq + (int64_t)g * 16 * d, &k_scale[g]);
+        else
+            quant_group(x, n * d, (uint8_t*)Kq + (int64_t)g * 16 * d, &k_scale[g]);
     }
     float* col = (float*)malloc((size_t)N * sizeof(float));
     uint8_t* cc = (uint8_t*)malloc((size_t)N);
@@ -563,6 +594,18 @@ void vo_sage_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_t*
     free(x);
     free(col);
     free(cc);
+}
+
+void vo_sage_quantize_head(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int N, int d,
+                           uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                           uint8_t* VcT, float* v_chscale, uint16_t* k_mean) {
+    sage_quantize(Q, K, V, N, d, Qq, q_scale, Kq, k_scale, VcT, v_chscale, k_mean, 0);
+}
+
+void vo_sage_quantize_head_i8(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int N, int d,
+                              int8_t* Qq, float* q_scale, int8_t* Kq, float* k_scale,
+                              uint8_t* VcT, float* v_chscale, uint16_t* k_mean) {
+    sage_quantize(Q, K, V, N, d, Qq, q_scale, Kq, k_scale, VcT, v_chscale, k_mean, 1);
 }
 
 /* --------------------------------------------------------------- attention */
@@ -796,10 +839,9 @@ void vo_attention_head_ex(const uint8_t* Qq, const float* q_scale, const uint8_t
 /* Attention on SAGE-style operands: the same row algorithm (ExpCast codes,
  * online reference) with per-token Q scales, per-16-key K scales, no V block
  * exponents or means, and output channel c multiplied by v_chscale[c]. */
-void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
-                            const float* k_scale, const uint8_t* VcT, const float* v_chscale,
-                            int N, int d, double softmax_scale, const int32_t* rows, int nrows,
-                            int flags, double* O, double* lse) {
+static void sage_attention(const void* Qq, const float* q_scale, const void* Kq, const float* k_scale,
+                           const uint8_t* VcT, const float* v_chscale, int N, int d, double softmax_scale,
+                           const int32_t* rows, int nrows, int flags, double* O, double* lse, int qk_i8) {
     int nb = (N + VO_BLOCK - 1) / VO_BLOCK;
     int64_t Np = (int64_t)nb * VO_BLOCK;
     double* qh = (double*)malloc((size_t)N * d * sizeof(double));
@@ -813,9 +855,10 @@ void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8
         qs[j] = q_scale[j];
         ks[j] = k_scale[j / 16];
         for (int c = 0; c < d; ++c) {
-            qh[(int64_t)j * d + c] = vo_e4m3_decode(Qq[(int64_t)j * d + c]);
-            kh[(int64_t)j * d + c] = vo_e4m3_decode(Kq[(int64_t)j * d + c]);
-            rh[(int64_t)j * d + c] = vo_e4m3_decode(VcT[(int64_t)c * Np + j]);
+            int64_t e = (int64_t)j * d + c;
+            qh[e] = qk_i8 ? (double)((const int8_t*)Qq)[e] : vo_e4m3_decode(((const uint8_t*)Qq)[e]);
+            kh[e] = qk_i8 ? (double)((const int8_t*)Kq)[e] : vo_e4m3_decode(((const uint8_t*)Kq)[e]);
+            rh[e] = vo_e4m3_decode(VcT[(int64_t)c * Np + j]);
         }
     }
     attn_rows(qh, qs, kh, ks, rh, ve, mu, N, d, softmax_scale, rows, nrows, flags, -INFINITY, O, lse, NULL, NULL,
@@ -823,6 +866,23 @@ void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8
     for (int r = 0; r < nrows; ++r)
         for (int c = 0; c < d; ++c) O[(int64_t)r * d + c] *= v_chscale[c];
     free(qh); free(kh); free(rh); free(qs); free(ks); free(mu); free(ve);
+}
+
+void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+                            const float* k_scale, const uint8_t* VcT, const float* v_chscale,
+                            int N, int d, double softmax_scale, const int32_t* rows, int nrows,
+                            int flags, double* O, double* lse) {
+    sage_attention(Qq, q_scale, Kq, k_scale, VcT, v_chscale, N, d, softmax_scale, rows, nrows, flags, O, lse, 0);
+}
+
+/* The same on INT8 Q and K' codes (vo_sage_quantize_head_i8): the code values
+ * are the integers themselves, so q.k is exact; z, the codes and the rest of
+ * the row algorithm are those of vo_attention_head_sage. */
+void vo_attention_head_sage_i8(const int8_t* Qq, const float* q_scale, const int8_t* Kq,
+                               const float* k_scale, const uint8_t* VcT, const float* v_chscale,
+                               int N, int d, double softmax_scale, const int32_t* rows, int nrows,
+                               int flags, double* O, double* lse) {
+    sage_attention(Qq, q_scale, Kq, k_scale, VcT, v_chscale, N, d, softmax_scale, rows, nrows, flags, O, lse, 1);
 }
 
 /* The 4-bit variant's probability step on its own: n <= 128 consecutive keys

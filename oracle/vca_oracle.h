@@ -133,6 +133,15 @@ void vo_attention_head_sage(const uint8_t* Qq, const float* q_scale, const uint8
                             const float* k_scale, const uint8_t* VcT, const float* v_chscale,
                             int N, int d, double softmax_scale, const int32_t* rows, int nrows,
                             int flags, double* O, double* lse);
+/* The post's INT8 qk_dtype: Q and K' groups as signed bytes, scale amax/127,
+ * code rne(x * (127/amax)) in fp32; V, k_mean and layouts as above. */
+void vo_sage_quantize_head_i8(const uint16_t* Q, const uint16_t* K, const uint16_t* V, int N, int d,
+                              int8_t* Qq, float* q_scale, int8_t* Kq, float* k_scale,
+                              uint8_t* VcT, float* v_chscale, uint16_t* k_mean);
+void vo_attention_head_sage_i8(const int8_t* Qq, const float* q_scale, const int8_t* Kq,
+                               const float* k_scale, const uint8_t* VcT, const float* v_chscale,
+                               int N, int d, double softmax_scale, const int32_t* rows, int nrows,
+                               int flags, double* O, double* lse);
 
 /* A second reading of the V residual scale: one exponent per head (v_exp[b] all
  * equal to it); everything else as vo_smooth_quantize_head. */
