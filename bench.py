@@ -322,7 +322,22 @@ def run_ours(args, world, rank, local):
 
         sage = {"prep_ms": round(g0.elapsed_time(g1) / 3, 3), "attn_ms": round(g1.elapsed_time(g2) / 3, 3),
                 "fidelity_vs_bf16_exact_softmax": {"v_smooth": fid(O_vc), "sage": fid(O_sg)}}
-        del sops, O_sg, O_vc, O_ex
+        del sops, O_sg
+        # the post's INT8 qk_dtype: Q/K as signed bytes, QK^T as kind::i8
+        iops = vca.sage_quantize(Q, K, V, ws=ws, qk_dtype="int8")
+        O_si = vca.attention_fwd_sage(iops, N, scale, ws=ws)
+        torch.cuda.synchronize()
+        g0.record(stream)
+        for _ in range(3):
+            vca.sage_quantize(Q, K, V, ws=ws, qk_dtype="int8")
+        g1.record(stream)
+        for _ in range(3):
+            vca.attention_fwd_sage(iops, N, scale, O=O_si, ws=ws)
+        g2.record(stream)
+        torch.cuda.synchronize()
+        sage["int8_qk"] = {"prep_ms": round(g0.elapsed_time(g1) / 3, 3), "attn_ms": round(g1.elapsed_time(g2) / 3, 3),
+                           "fidelity_vs_bf16_exact_softmax": fid(O_si)}
+        del iops, O_si, O_vc, O_ex
         ws.check()
 
     # ---- end to end through the C ABI with host buffers: vca_vc_attention_host

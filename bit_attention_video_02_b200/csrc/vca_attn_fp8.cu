@@ -110,7 +110,9 @@ __device__ __forceinline__ uint32_t tf32_tile_off(int r, int k) {
 // SAGE: operands of the SAGE-style comparison recipe (vca_sage_quantize_qkv):
 // one Q scale per token, one K scale per 16 keys, V with per-channel scales
 // applied to the output and no block exponents or means (no mean restore).
-template <bool SKIP, bool SAGE>
+// QI8 (SAGE only): Q and K are INT8 codes, QK^T runs as kind::i8 into s32
+// accumulators, converted exactly to fp32 (|q.k| < 2^21) after the load.
+template <bool SKIP, bool SAGE, bool QI8 = false>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -194,7 +196,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     // each tcgen05 instruction.  (The issuing warp shares its SM sub-partition
     // with two softmax warps: the fewer instructions per MMA, the sooner the
     // tensor pipe gets its next operation.)
-    const uint32_t id_qk = instr_desc(kFmtE4M3, kFmtE4M3, 128, 128, 0, 0);
+    const uint32_t id_qk = QI8 ? instr_desc_s8(128, 128) : instr_desc(kFmtE4M3, kFmtE4M3, 128, 128, 0, 0);
     const uint32_t id_pv = instr_desc_mx(kFmtE4M3, kFmtE4M3, 128, 128);
     const uint32_t id_mu = instr_desc(kFmtTF32, kFmtTF32, 128, 128, 0, 0);
     // descriptor start addresses count 16-byte units: +2 per 32-byte K step,
@@ -210,8 +212,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     auto issue_qk = [&](int t, int jj) {
       const int s1 = jj % kStages;
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_f8_ss_w(tS, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(s1 * 1024 + 2 * k), id_qk, k > 0);
+      for (int k = 0; k < 4; ++k) {
+        if (QI8)
+          mma_i8_ss_w(tS, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(s1 * 1024 + 2 * k), id_qk, k > 0);
+        else
+          mma_f8_ss_w(tS, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(s1 * 1024 + 2 * k), id_qk, k > 0);
+      }
       tc_commit_w(&bars.s_full[t]);
     };
     // O_t += P_t(j) R_j 2^e_j, and at a group end the mean restore of the group;
@@ -374,6 +380,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       // the scores are in registers: S may take the other tile's next scores
       tc_fence_before();
       mbar_arrive(&bars.s_free[t]);
+      if (QI8) {
+        // s32 -> fp32 exactly: the integer sits in the mantissa of 1.5 * 2^23
+        uint32_t* su = reinterpret_cast<uint32_t*>(sv);
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float2 f = __fadd2_rn(make_float2(__uint_as_float(su[c] + 0x4B400000u),
+                                                  __uint_as_float(su[c + 1] + 0x4B400000u)),
+                                      make_float2(-kMagic, -kMagic));
+          sv[c] = f.x;
+          sv[c + 1] = f.y;
+        }
+      }
       const int valid = min(128, N - j * 128);
       if (valid < 128) {
 #pragma unroll
@@ -574,11 +592,12 @@ using namespace vca;
 
 extern "C" size_t vca_attention_workspace_size(int B, int H, int N) { return 256; }
 
-static int attention_launch(const char* fn, const uint8_t* Qq, const float* q_scale, const uint8_t* Kq,
+static int attention_launch(const char* fn, const void* Qq, const float* q_scale, const void* Kq,
                             const float* k_scale, const uint8_t* VrT, const int8_t* v_exp,
                             const vca_bf16* v_mean, int B, int H, int N, int d, float softmax_scale,
                             vca_bf16* O, float* lse, void* ws, size_t ws_bytes, float skip_lambda,
-                            unsigned long long* skipped, const float* v_chscale, vca_stream_t stream) {
+                            unsigned long long* skipped, const float* v_chscale, vca_stream_t stream,
+                            bool qk_i8 = false) {
   const bool sage = v_chscale != nullptr;   // SAGE operands: no V exponents or means
   if (d != VCA_HEAD_DIM) return fail(VCA_ERR_UNSUPPORTED, "%s: d must be 128", fn);
   if (B < 1 || H < 1 || N < 1 || (int64_t)B * H > 65535)
@@ -627,7 +646,11 @@ static int attention_launch(const char* fn, const uint8_t* Qq, const float* q_sc
   prm.skipped = skipped;
   prm.v_chscale = v_chscale;
   if (skip && sage) return fail(VCA_ERR_UNSUPPORTED, "%s: Skip Softmax on SAGE operands is not built", fn);
-  auto kern = skip ? attn_fp8_kernel<true, false> : sage ? attn_fp8_kernel<false, true> : attn_fp8_kernel<false, false>;
+  if (qk_i8 && !sage) return fail(VCA_ERR_UNSUPPORTED, "%s: INT8 QK^T is built for SAGE operands only", fn);
+  auto kern = skip    ? attn_fp8_kernel<true, false>
+              : qk_i8 ? attn_fp8_kernel<false, true, true>
+              : sage  ? attn_fp8_kernel<false, true>
+                      : attn_fp8_kernel<false, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemAlloc) != cudaSuccess)
     return fail(VCA_ERR_CUDA, "%s: cannot set shared-memory size", fn);
   dim3 grid((nb + 1) / 2, (unsigned)BH);
@@ -661,4 +684,13 @@ extern "C" int vca_attention_fwd_sage(const uint8_t* Qq, const float* q_scale, c
   if (!v_chscale) return fail(VCA_ERR_INVALID, "vca_attention_fwd_sage: null pointer");
   return attention_launch("vca_attention_fwd_sage", Qq, q_scale, Kq, k_scale, VcT, nullptr, nullptr, B, H, N, d,
                           softmax_scale, O, lse, ws, ws_bytes, 0.0f, nullptr, v_chscale, stream);
+}
+
+extern "C" int vca_attention_fwd_sage_i8(const int8_t* Qq, const float* q_scale, const int8_t* Kq,
+                                         const float* k_scale, const uint8_t* VcT, const float* v_chscale, int B,
+                                         int H, int N, int d, float softmax_scale, vca_bf16* O, float* lse,
+                                         void* ws, size_t ws_bytes, vca_stream_t stream) {
+  if (!v_chscale) return fail(VCA_ERR_INVALID, "vca_attention_fwd_sage_i8: null pointer");
+  return attention_launch("vca_attention_fwd_sage_i8", Qq, q_scale, Kq, k_scale, VcT, nullptr, nullptr, B, H, N,
+                          d, softmax_scale, O, lse, ws, ws_bytes, 0.0f, nullptr, v_chscale, stream, true);
 }

@@ -157,6 +157,13 @@ __device__ __forceinline__ void mma_f8_ss_w(uint32_t d, uint64_t a, uint64_t b, 
       "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(accum));
 }
+__device__ __forceinline__ void mma_i8_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                            uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accum));
+}
 __device__ __forceinline__ void mma_mxf8_ts_w(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
                                               uint32_t sfa, uint32_t sfb, uint32_t accum) {
   asm volatile(
@@ -265,6 +272,11 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t afmt, uint32_t bfmt, 
                                                   uint32_t a_mn_major, uint32_t b_mn_major) {
   return (1u << 4) | (afmt << 7) | (bfmt << 10) | (a_mn_major << 15) | (b_mn_major << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// Integer kind (kind::i8): D format 2 (s32) in [4,6), A and B type 1 (signed
+// 8-bit), no saturation (|sum| < 2^21 for 128 products of magnitude <= 127^2).
+__host__ __device__ constexpr uint32_t instr_desc_s8(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 // Block-scaled variant (kind::mxf8f6f4): B scale-factor id in [4,6), scale
 // format bit 23 (1 = UE8M0), A scale-factor id in [29,31); no D-format field.

@@ -11,6 +11,9 @@
 //               stored channel-major (VcT [d][Np]) like V-Smooth's residual
 // No reordering and no block means: this is the recipe V-Smooth is compared to.
 //
+// qk_dtype int8 (the post's other choice, and the one it runs): Q and K' as
+// signed bytes, amax/127 and rne(x * 127/amax), same groups; V stays E4M3.
+//
 // Three launches: channel statistics (exact K sums, V maxima), a tiny finalise
 // (k_mean, per-channel V scales), and the quantisation of 128-token blocks.
 #include "vca_device.cuh"
@@ -95,7 +98,33 @@ struct SageArgs {
   uint8_t* Kq;
   float* k_scale;    // [BH][Np/16]
   uint8_t* VcT;      // [BH][128][Np]
+  int qk_i8;         // Q and K' as INT8 (amax/127, rne) instead of E4M3 (amax/448)
 };
+
+// Four fp32 values (already multiplied by 127/amax) as signed bytes, round to
+// nearest even, in [-127, 127].
+__device__ __forceinline__ uint32_t cvt_s8x4(float a, float b, float c, float d) {
+  const int v[4] = {__float2int_rn(a), __float2int_rn(b), __float2int_rn(c), __float2int_rn(d)};
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w |= (uint32_t)(min(127, max(-127, v[i])) & 0xFF) << (8 * i);
+  return w;
+}
+
+// Eight codes of one thread's channels: x * inv rounded once in fp32, then
+// coded as E4M3 (cvt, RNE, saturating) or as signed bytes.
+__device__ __forceinline__ void c2_codes(const float (&x)[8], float inv, int qk_i8, uint32_t (&c2)[2]) {
+  float y[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) y[c] = __fmul_rn(x[c], inv);
+  if (qk_i8) {
+    c2[0] = cvt_s8x4(y[0], y[1], y[2], y[3]);
+    c2[1] = cvt_s8x4(y[4], y[5], y[6], y[7]);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) c2[q >> 1] |= (uint32_t)cvt_e4m3x2(y[2 * q], y[2 * q + 1]) << ((q & 1) * 16);
+  }
+}
 
 // One CTA per (128-token block, tensor, head).  Thread t holds the 8 channels
 // 8*(t%16).. of token rows 16*it + t/16 (it = 0..7), as 16-byte loads; the 16
@@ -135,16 +164,12 @@ __global__ void __launch_bounds__(kSageThreads) sage_quant_kernel(const SageArgs
 #pragma unroll
       for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       const bool live = row < nv && m > 0.0f;
-      const float inv = live ? __fdiv_rn(448.0f, m) : 0.0f;
+      const float qmax = a.qk_i8 ? 127.0f : 448.0f;
+      const float inv = live ? __fdiv_rn(qmax, m) : 0.0f;
       uint32_t c2[2] = {0u, 0u};
-      if (live) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          c2[q >> 1] |= (uint32_t)cvt_e4m3x2(__fmul_rn(x[it][2 * q], inv), __fmul_rn(x[it][2 * q + 1], inv))
-                        << ((q & 1) * 16);
-      }
+      if (live) c2_codes(x[it], inv, a.qk_i8, c2);
       *reinterpret_cast<uint2*>(dst + (int64_t)row * 128 + chunk * 8) = make_uint2(c2[0], c2[1]);
-      if (chunk == 0) a.q_scale[(int64_t)bh * Np + n0 + row] = live ? __fdiv_rn(m, 448.0f) : 1.0f;
+      if (chunk == 0) a.q_scale[(int64_t)bh * Np + n0 + row] = live ? __fdiv_rn(m, qmax) : 1.0f;
     }
     return;
   }
@@ -178,15 +203,13 @@ __global__ void __launch_bounds__(kSageThreads) sage_quant_kernel(const SageArgs
       float m = red[0][it];
 #pragma unroll
       for (int w = 1; w < kSageThreads / 32; ++w) m = fmaxf(m, red[w][it]);
-      const float inv = m > 0.0f ? __fdiv_rn(448.0f, m) : 0.0f;
+      const float qmax = a.qk_i8 ? 127.0f : 448.0f;
+      const float inv = m > 0.0f ? __fdiv_rn(qmax, m) : 0.0f;
       const int row = it * 16 + rsub;
       uint32_t c2[2] = {0u, 0u};
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        c2[q >> 1] |= (uint32_t)cvt_e4m3x2(__fmul_rn(x[it][2 * q], inv), __fmul_rn(x[it][2 * q + 1], inv))
-                      << ((q & 1) * 16);
+      c2_codes(x[it], inv, a.qk_i8, c2);
       *reinterpret_cast<uint2*>(dst + (int64_t)row * 128 + chunk * 8) = make_uint2(c2[0], c2[1]);
-      if (t == 0) a.k_scale[(int64_t)bh * (Np / 16) + blk * 8 + it] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
+      if (t == 0) a.k_scale[(int64_t)bh * (Np / 16) + blk * 8 + it] = m > 0.0f ? __fdiv_rn(m, qmax) : 1.0f;
     }
     return;
   }
@@ -228,11 +251,10 @@ extern "C" size_t vca_sage_quantize_workspace_size(int B, int H, int N) {
   return total;
 }
 
-extern "C" int vca_sage_quantize_qkv(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V, int B, int H,
-                                     int N, int d, uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
-                                     uint8_t* VcT, float* v_chscale, vca_bf16* k_mean, void* ws,
-                                     size_t ws_bytes, vca_stream_t stream) {
-  const char* fn = "vca_sage_quantize_qkv";
+static int sage_quantize(const char* fn, const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V, int B, int H,
+                         int N, int d, void* Qq, float* q_scale, void* Kq, float* k_scale, uint8_t* VcT,
+                         float* v_chscale, vca_bf16* k_mean, void* ws, size_t ws_bytes, int qk_i8,
+                         vca_stream_t stream) {
   if (d != VCA_HEAD_DIM) return fail(VCA_ERR_UNSUPPORTED, "%s: d must be 128", fn);
   if (B < 1 || H < 1 || N < 1 || (int64_t)B * H > 65535 || N > (1 << 24))
     return fail(VCA_ERR_INVALID, "%s: bad shape B=%d H=%d N=%d", fn, B, H, N);
@@ -257,7 +279,24 @@ extern "C" int vca_sage_quantize_qkv(const vca_bf16* Q, const vca_bf16* K, const
   if ((rc = check_launch("sage_finalize_kernel"))) return rc;
   SageArgs a;
   a.Q = Q; a.K = K; a.V = V; a.k_mean = k_mean; a.vinv = w.vinv; a.N = N; a.nb = (N + 127) / 128;
-  a.Qq = Qq; a.q_scale = q_scale; a.Kq = Kq; a.k_scale = k_scale; a.VcT = VcT;
+  a.Qq = (uint8_t*)Qq; a.q_scale = q_scale; a.Kq = (uint8_t*)Kq; a.k_scale = k_scale; a.VcT = VcT;
+  a.qk_i8 = qk_i8;
   sage_quant_kernel<<<dim3(a.nb, 3, BH), kSageThreads, 0, s>>>(a);
   return check_launch("sage_quant_kernel");
+}
+
+extern "C" int vca_sage_quantize_qkv(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V, int B, int H,
+                                     int N, int d, uint8_t* Qq, float* q_scale, uint8_t* Kq, float* k_scale,
+                                     uint8_t* VcT, float* v_chscale, vca_bf16* k_mean, void* ws,
+                                     size_t ws_bytes, vca_stream_t stream) {
+  return sage_quantize("vca_sage_quantize_qkv", Q, K, V, B, H, N, d, Qq, q_scale, Kq, k_scale, VcT, v_chscale,
+                       k_mean, ws, ws_bytes, 0, stream);
+}
+
+extern "C" int vca_sage_quantize_qkv_i8(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V, int B, int H,
+                                        int N, int d, int8_t* Qq, float* q_scale, int8_t* Kq, float* k_scale,
+                                        uint8_t* VcT, float* v_chscale, vca_bf16* k_mean, void* ws,
+                                        size_t ws_bytes, vca_stream_t stream) {
+  return sage_quantize("vca_sage_quantize_qkv_i8", Q, K, V, B, H, N, d, Qq, q_scale, Kq, k_scale, VcT, v_chscale,
+                       k_mean, ws, ws_bytes, 1, stream);
 }

@@ -35,6 +35,7 @@ EXPORTED = [
     "vca_bf16_attention_workspace_size", "vca_bf16_attention_fwd", "vca_schedule_regroup",
     "vca_attention_fwd_skip", "vca_vc_attention_host_buffer_size", "vca_vc_attention_host",
     "vca_sage_quantize_workspace_size", "vca_sage_quantize_qkv", "vca_attention_fwd_sage",
+    "vca_sage_quantize_qkv_i8", "vca_attention_fwd_sage_i8",
     "vca_smooth_quantize_fp4_workspace_size", "vca_smooth_quantize_qkv_fp4",
     "vca_attention_fwd_fp4", "vca_debug_fp4_mma",
 ]
@@ -80,6 +81,8 @@ def lib() -> ctypes.CDLL:
         L.vca_sage_quantize_workspace_size.argtypes = [i32, i32, i32]
         L.vca_sage_quantize_qkv.argtypes = [vp, vp, vp] + [i32] * 4 + [vp] * 7 + [vp, sz, vp]
         L.vca_attention_fwd_sage.argtypes = [vp] * 6 + [i32] * 4 + [f32, vp, vp, vp, sz, vp]
+        L.vca_sage_quantize_qkv_i8.argtypes = L.vca_sage_quantize_qkv.argtypes
+        L.vca_attention_fwd_sage_i8.argtypes = L.vca_attention_fwd_sage.argtypes
         L.vca_smooth_quantize_fp4_workspace_size.restype = sz
         L.vca_smooth_quantize_fp4_workspace_size.argtypes = [i32, i32, i32]
         L.vca_smooth_quantize_qkv_fp4.argtypes = [vp] * 4 + [i32] * 4 + [vp] * 8 + [vp, sz, vp]
@@ -93,7 +96,7 @@ def lib() -> ctypes.CDLL:
                    "vca_smooth_quantize_qkv",
                    "vca_attention_fwd", "vca_bf16_attention_fwd", "vca_schedule_regroup",
                    "vca_attention_fwd_skip", "vca_vc_attention_host", "vca_sage_quantize_qkv",
-                   "vca_attention_fwd_sage"):
+                   "vca_attention_fwd_sage", "vca_sage_quantize_qkv_i8", "vca_attention_fwd_sage_i8"):
             getattr(L, fn).restype = i32
         _lib = L
     return _lib
@@ -391,22 +394,28 @@ def vc_attention_host(Q, K, V, k: int = 32, iters: int = 3, softmax_scale=None, 
     return O
 
 
-def sage_quantize(Q, K, V, ws: Workspace | None = None, stream=None) -> dict:
-    """vca_sage_quantize_qkv: the SAGE-style comparison quantisation."""
+def sage_quantize(Q, K, V, ws: Workspace | None = None, stream=None, qk_dtype: str = "fp8") -> dict:
+    """vca_sage_quantize_qkv (qk_dtype "fp8": E4M3 Q and K') or
+    vca_sage_quantize_qkv_i8 ("int8": signed-byte Q and K'): the SAGE-style
+    comparison quantisation."""
+    if qk_dtype not in ("fp8", "int8"):
+        raise ValueError(f"qk_dtype must be 'fp8' or 'int8', not {qk_dtype!r}")
     B, H, N, d = _bhnd(Q)
     dev = Q.device
     nb = (N + 127) // 128
     Np = nb * 128
-    out = dict(Qq=torch.empty(B, H, Np, d, dtype=torch.uint8, device=dev),
+    ct = torch.int8 if qk_dtype == "int8" else torch.uint8
+    out = dict(Qq=torch.empty(B, H, Np, d, dtype=ct, device=dev),
                q_scale=torch.empty(B, H, Np, dtype=torch.float32, device=dev),
-               Kq=torch.empty(B, H, Np, d, dtype=torch.uint8, device=dev),
+               Kq=torch.empty(B, H, Np, d, dtype=ct, device=dev),
                k_scale=torch.empty(B, H, Np // 16, dtype=torch.float32, device=dev),
                VcT=torch.empty(B, H, d, Np, dtype=torch.uint8, device=dev),
                v_chscale=torch.empty(B, H, d, dtype=torch.float32, device=dev),
                k_mean=torch.empty(B, H, d, dtype=torch.bfloat16, device=dev))
     need = lib().vca_sage_quantize_workspace_size(B, H, N)
     ws = (ws or Workspace(need, dev)).ensure(need)
-    _check(lib().vca_sage_quantize_qkv(
+    fn = lib().vca_sage_quantize_qkv_i8 if qk_dtype == "int8" else lib().vca_sage_quantize_qkv
+    _check(fn(
         _ptr(Q), _ptr(K), _ptr(V), B, H, N, d, _ptr(out["Qq"]), _ptr(out["q_scale"]), _ptr(out["Kq"]),
         _ptr(out["k_scale"]), _ptr(out["VcT"]), _ptr(out["v_chscale"]), _ptr(out["k_mean"]), ws.ptr, ws.nbytes,
         _stream(stream)))
@@ -448,8 +457,12 @@ def debug_fp4_mma(a_codes, sf_cols, b_codes, ws: Workspace | None = None, stream
 
 def attention_fwd_sage(ops: dict, N: int, softmax_scale: float | None = None, O=None, lse=None,
                        want_lse: bool = False, ws: Workspace | None = None, stream=None):
-    """vca_attention_fwd_sage: FP8 attention on SAGE-style operands."""
+    """vca_attention_fwd_sage (E4M3 Q/K) or vca_attention_fwd_sage_i8 (int8 Q/K,
+    picked by the operands' dtype): attention on SAGE-style operands."""
     B, H, Np, d = ops["Qq"].shape
+    if ops["Qq"].dtype != ops["Kq"].dtype or ops["Qq"].dtype not in (torch.uint8, torch.int8):
+        raise ValueError("Qq and Kq must both be uint8 (E4M3) or both int8")
+    fn = lib().vca_attention_fwd_sage_i8 if ops["Qq"].dtype == torch.int8 else lib().vca_attention_fwd_sage
     scale = 1.0 / math.sqrt(d) if softmax_scale is None else float(softmax_scale)
     dev = ops["Qq"].device
     if O is None:
@@ -458,7 +471,7 @@ def attention_fwd_sage(ops: dict, N: int, softmax_scale: float | None = None, O=
         lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
     need = lib().vca_attention_workspace_size(B, H, N)
     ws = (ws or Workspace(need, dev)).ensure(need)
-    _check(lib().vca_attention_fwd_sage(
+    _check(fn(
         _ptr(ops["Qq"]), _ptr(ops["q_scale"]), _ptr(ops["Kq"]), _ptr(ops["k_scale"]), _ptr(ops["VcT"]),
         _ptr(ops["v_chscale"]), B, H, N, d, scale, _ptr(O), _ptr(lse), ws.ptr, ws.nbytes, _stream(stream)))
     return (O, lse) if want_lse else O

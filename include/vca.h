@@ -353,6 +353,25 @@ int vca_attention_fwd_sage(const uint8_t* Qq, const float* q_scale, const uint8_
                            float softmax_scale, vca_bf16* O, float* lse, void* ws, size_t ws_bytes,
                            vca_stream_t stream);
 
+/* The post's other qk_dtype, INT8 (the one it runs), on the same recipe:
+ *   Qq, Kq int8 [B][H][Np][d]; q_scale = max|x| / 127 per token, k_scale the
+ *   same per 16 smoothed keys; codes rne(x * (127 / max|x|)) with the product
+ *   in fp32, in [-127, 127]; an all-zero group has scale 1 and codes 0.
+ * V (E4M3, per channel), k_mean, padding, workspace and errors exactly as
+ * vca_sage_quantize_qkv. */
+int vca_sage_quantize_qkv_i8(const vca_bf16* Q, const vca_bf16* K, const vca_bf16* V, int B, int H, int N, int d,
+                             int8_t* Qq, float* q_scale, int8_t* Kq, float* k_scale, uint8_t* VcT,
+                             float* v_chscale, vca_bf16* k_mean, void* ws, size_t ws_bytes, vca_stream_t stream);
+
+/* vca_attention_fwd_sage on the INT8 operands of vca_sage_quantize_qkv_i8:
+ * QK^T is a tcgen05 kind::i8 MMA with s32 accumulation (exact: |q.k| < 2^21),
+ * converted exactly to fp32 before z = s * q_scale * k_scale * softmax_scale *
+ * log2(e); everything after that as vca_attention_fwd_sage. */
+int vca_attention_fwd_sage_i8(const int8_t* Qq, const float* q_scale, const int8_t* Kq, const float* k_scale,
+                              const uint8_t* VcT, const float* v_chscale, int B, int H, int N, int d,
+                              float softmax_scale, vca_bf16* O, float* lse, void* ws, size_t ws_bytes,
+                              vca_stream_t stream);
+
 /* In-repo BF16 comparator: exact-softmax flash attention (online softmax with
  * exp2), tcgen05 BF16 MMAs with fp32 accumulation in tensor memory.
  *   Q, K, V, O [B][H][N][d] bf16; lse [B][H][N] fp32 natural log (nullable). */
