@@ -52,7 +52,9 @@ constexpr int kGroup = 8;   // key blocks per mean-restore MMA
 
 // TMEM columns
 constexpr uint32_t kColS = 0;     // score tile (128 columns)
-constexpr uint32_t kColP = 128;   // P region: tile t at +64t: scale vectors +0..+7, codes +8..+39
+constexpr uint32_t kColP = 128;   // P region: tile t at +64t: scale vectors +0..+7, codes +8..+39,
+                                  // block row sum (16-column MMA output, column 0 used) +48..+63
+constexpr uint32_t kColRowSum = 48;
 constexpr uint32_t kColO = 256;   // O_t at +128t
 
 // dynamic shared memory layout (offsets from a 1024-aligned base)
@@ -61,7 +63,8 @@ constexpr uint32_t kOffK = 32768;                     // kStages x 16 KB
 constexpr uint32_t kOffV = kOffK + kStages * 16384;   // kStages x 16 KB
 constexpr uint32_t kOffL = kOffV + kStages * 16384;   // 2 tiles x (hi 4 KB + lo 4 KB)
 constexpr uint32_t kOffMu = kOffL + 16384;            // 2 buffers x 4 KB
-constexpr uint32_t kSmemBytes = kOffMu + 8192;
+constexpr uint32_t kOffOnes = kOffMu + 8192;          // 16 x 32 E4M3: row 0 ones, rows 1-15 zero
+constexpr uint32_t kSmemBytes = kOffOnes + 1024;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 
 struct AttnParams {
@@ -112,6 +115,14 @@ __device__ __forceinline__ uint32_t tf32_tile_off(int r, int k) {
 // applied to the output and no block exponents or means (no mean restore).
 // QI8 (SAGE only): Q and K are INT8 codes, QK^T runs as kind::i8 into s32
 // accumulators, converted exactly to fp32 (|q.k| < 2^21) after the load.
+// block row sum l -> L tile entry (row r, block kk of the group): the hi part
+// exact in TF32, lo the remainder
+__device__ __forceinline__ void store_l(uint8_t* sLt, int r, int kk, float l) {
+  const float hi = __uint_as_float(__float_as_uint(l) & 0xFFFFE000u);
+  *reinterpret_cast<float*>(sLt + tf32_tile_off(r, kk)) = hi;
+  *reinterpret_cast<float*>(sLt + 4096 + tf32_tile_off(r, kk)) = l - hi;
+}
+
 template <bool SKIP, bool SAGE, bool QI8 = false>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -151,6 +162,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     tma_prefetch_desc(&p.tmQ);
     tma_prefetch_desc(&p.tmK);
     tma_prefetch_desc(&p.tmV);
+  }
+  // the row-sum operand: B [16 x 32] K-major, no swizzle (core matrices of 8
+  // rows x 16 bytes, 128 bytes apart along K, 256 apart along N); row 0 holds
+  // E4M3 1.0 (0x38), rows 1-15 zero.  Every K step of the row-sum MMA reads it.
+  if (threadIdx.x < 128) {
+    const int off = threadIdx.x * 4;   // 512 bytes
+    const int in_cm = off & 127;       // byte within a core matrix: row (in_cm / 16)
+    const bool row0 = (off < 256) && (in_cm < 16);
+    *reinterpret_cast<uint32_t*>(sm + kOffOnes + off) = row0 ? 0x38383838u : 0u;
+    fence_proxy_async_smem();
   }
   // a CTA of this launch (or of an earlier one sharing the workspace) already
   // timed out: do no work, so a broken pipeline costs one wait, not one per CTA
@@ -199,6 +220,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const uint32_t id_qk = QI8 ? instr_desc_s8(128, 128) : instr_desc(kFmtE4M3, kFmtE4M3, 128, 128, 0, 0);
     const uint32_t id_pv = instr_desc_mx(kFmtE4M3, kFmtE4M3, 128, 128);
     const uint32_t id_mu = instr_desc(kFmtTF32, kFmtTF32, 128, 128, 0, 0);
+    const uint32_t id_rs = instr_desc(kFmtE4M3, kFmtE4M3, 128, 16, 0, 0);
+    const uint64_t dOnes = smem_desc(smem_u32(sm + kOffOnes), 128, 256, kLayoutNone);
     // descriptor start addresses count 16-byte units: +2 per 32-byte K step,
     // +1024 per 16 KB tile, +256 per 4 KB
     const uint64_t dQ = smem_desc(smem_u32(sm + kOffQ), 16, 1024, kLayoutSW128);
@@ -220,8 +243,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       }
       tc_commit_w(&bars.s_full[t]);
     };
-    // O_t += P_t(j) R_j 2^e_j, and at a group end the mean restore of the group;
-    // o_done[t] then tracks everything that reads the P region or writes O_t
+    // mean restore of group g: O_t += L_t(g) M(g) (L split hi + lo); after
+    // tile 1's, the block-mean buffer may be refilled
+    auto issue_mu = [&](int t, int g) -> bool {
+      const int gb = g & 1;
+      if (!mbar_wait_warp(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220)) return false;
+      tc_fence_after();
+      const uint64_t bdesc = dMu + (uint64_t)(gb * 256);
+      mma_tf32_ss_w(tmem + kColO + t * 128, dL + (uint64_t)(t * 512), bdesc, id_mu, 1u);
+      mma_tf32_ss_w(tmem + kColO + t * 128, dL + (uint64_t)(t * 512 + 256), bdesc, id_mu, 1u);
+      if (t == 1) tc_commit_w(&bars.mu_empty[gb]);
+      return true;
+    };
+    // O_t += P_t(j) R_j 2^e_j and the block row sums P_t(j) 1 (into the P
+    // region); the L tile of a group is complete once the warpgroup has read
+    // the row sums of its last block, so a group's mean restore is issued with
+    // the next group's first PV (the last group's after the loop).  o_done[t]
+    // then tracks everything that reads the P region or writes O_t.
     auto issue_pv = [&](int t, int j) -> bool {
       if (!mbar_wait_warp(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t)) return false;
       tc_fence_after();
@@ -234,22 +272,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         skip_pv = f[0] && f[1] && f[2] && f[3];
         nskip += skip_pv ? 1 : 0;
       }
+      if (!SAGE && j > 0 && j % kGroup == 0 && !issue_mu(t, j / kGroup - 1)) return false;
       if (!skip_pv) {
 #pragma unroll
         for (int k = 0; k < 4; ++k)   // 8 columns (32 codes) per K step
           mma_mxf8_ts_w(tmem + kColO + t * 128, tP + 8 + 8 * k, dV + (uint64_t)(s * 1024 + 2 * k), id_pv, tP,
                         tP + 4, (j > 0 || k > 0) ? 1u : 0u);
       }
-      const bool group_end = (j % kGroup == kGroup - 1) || (j == nkv - 1);
-      if (group_end && !SAGE) {
-        const int g = j / kGroup, gb = g & 1;
-        if (!mbar_wait_warp(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220)) return false;
-        tc_fence_after();
-        const uint64_t bdesc = dMu + (uint64_t)(gb * 256);
-        mma_tf32_ss_w(tmem + kColO + t * 128, dL + (uint64_t)(t * 512), bdesc, id_mu, 1u);
-        mma_tf32_ss_w(tmem + kColO + t * 128, dL + (uint64_t)(t * 512 + 256), bdesc, id_mu, 1u);
-        if (t == 1) tc_commit_w(&bars.mu_empty[gb]);
-      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)   // row sums: the same codes against a column of ones
+        mma_f8_ts_w(tP + kColRowSum, tP + 8 + 8 * k, dOnes, id_rs, k > 0 ? 1u : 0u);
+      tc_commit_w(&bars.o_done[t]);
+      return true;
+    };
+    // after the last block: the warpgroup has added the last row sums to the
+    // L tile; the last group's mean restore completes O_t
+    auto issue_last = [&](int t) -> bool {
+      if (!mbar_wait_warp(&bars.p_full[t], nkv & 1, &abort_s, p.st, lim, 240 + t)) return false;
+      tc_fence_after();
+      if (!SAGE && !issue_mu(t, (nkv - 1) / kGroup)) return false;
       tc_commit_w(&bars.o_done[t]);
       return true;
     };
@@ -293,6 +334,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         issue_qk(0, j + 2);
       }
     }
+    ok = ok && issue_last(0);
+    ok = ok && issue_last(1);
     tc_commit_w(&bars.mma_done);
     if (SKIP && lane == 0 && p.skipped && nskip) atomicAdd(p.skipped, nskip);
   } else if (warp == 2 && !SAGE) {
@@ -321,6 +364,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const uint32_t tS = tmem + kColS + lane_off;
     const uint32_t tP = tmem + kColP + t * 64 + lane_off;   // scale vectors +0..+7, codes +8..+39
     const uint32_t tO = tmem + kColO + t * 128 + lane_off;
+    const uint32_t tRS = tP + kColRowSum;          // this row's block row sum (column 0)
     const int qtile = pair * 2 + t;
     const bool qvalid = qtile < nb;
     const bool row_valid = qvalid && qtile * 128 + r < N;
@@ -450,22 +494,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         rescale = delta > 126 ? 0.0f : __uint_as_float((uint32_t)(127 - delta) << 23);
       }
       // ExpCast: code = rne(s*c8 + 87 - 8*nref) via the magic-number FMA (two
-      // scores per fma.rn.f32x2), clamped below at 0; the decoded probability is
-      // float(code << 20) * 2^120, summed exactly enough in fp32 pairs
+      // scores per fma.rn.f32x2), clamped below at 0; the block's row sum of the
+      // decoded probabilities comes from the tensor core (the codes against a
+      // column of ones), read one block later
       const bool warp_drop = SKIP && __all_sync(0xffffffffu, rej);
       // a dropped row writes code 0 everywhere: multiplier 0, addend the bare magic constant
       const float badd = rej ? kMagic : kMagic + (float)(87 - 8 * nref);
       const float c8r = rej ? 0.0f : c8;
       const float2 c8x2 = make_float2(c8r, c8r), baddx2 = make_float2(badd, badd);
-      float2 lsa = make_float2(0.0f, 0.0f), lsb = make_float2(0.0f, 0.0f);
       uint32_t pw[32];   // the row's 128 codes, 4 per word, in key order
-      // PV_t(j-1) (and the mean restore before it) must have completed before
-      // the P region, sL_t or O_t are written; it was issued when this
-      // warpgroup finished the previous block, so this wait rarely blocks
+      // PV_t(j-1), its row sums (and any mean restore before it) must have
+      // completed before the P region, sL_t or O_t are written; they were
+      // issued when this warpgroup finished the previous block, so this wait
+      // rarely blocks.  The row sum of block j-1 is loaded here and used after
+      // the code pass.
+      uint32_t lprev_bits = 0;
       if (j > 0) {
         ok = mbar_wait_warp(&bars.o_done[t], (j - 1) & 1, &abort_s, p.st, lim, 410 + t);
         if (!ok) break;
         tc_fence_after();
+        lprev_bits = tmem_ld1(tRS);
       }
       if (warp_drop) {
         // PV may still run for the other warps' rows: these rows contribute zeros
@@ -481,27 +529,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         const float2 f23 = __ffma2_rn(make_float2(sv[c + 2], sv[c + 3]), cx, baddx2);
         const uint32_t b0 = __float_as_uint(fmaxf(f01.x, kMagic)), b1 = __float_as_uint(fmaxf(f01.y, kMagic));
         const uint32_t b2 = __float_as_uint(fmaxf(f23.x, kMagic)), b3 = __float_as_uint(fmaxf(f23.y, kMagic));
-        lsa = __fadd2_rn(lsa, make_float2(__uint_as_float(b0 << 20), __uint_as_float(b1 << 20)));
-        lsb = __fadd2_rn(lsb, make_float2(__uint_as_float(b2 << 20), __uint_as_float(b3 << 20)));
         pw[q] = prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
       }
       VCA_TMEM_ST32(tP + 8, pw);
       }
-      const float lsum = (lsa.x + lsa.y) + (lsb.x + lsb.y);
-      const float l = lsum * 0x1p120f;
-      // block row sum -> L tile (hi part exact in TF32, lo the remainder)
-      if (!SAGE) {
-        const int kk = j % kGroup;
-        const float hi = __uint_as_float(__float_as_uint(l) & 0xFFFFE000u);
-        const float lo = l - hi;
-        *reinterpret_cast<float*>(sLt + tf32_tile_off(r, kk)) = hi;
-        *reinterpret_cast<float*>(sLt + 4096 + tf32_tile_off(r, kk)) = lo;
-        if (j == nkv - 1) {
-          for (int k2 = kk + 1; k2 < kGroup; ++k2) {
-            *reinterpret_cast<float*>(sLt + tf32_tile_off(r, k2)) = 0.0f;
-            *reinterpret_cast<float*>(sLt + 4096 + tf32_tile_off(r, k2)) = 0.0f;
-          }
-        }
+      if (j > 0) {
+        // block j-1's row sum (in the units of the reference before this
+        // block's rescale) -> L tile and the running total
+        tmem_ld_wait();
+        reg_after_wait(lprev_bits);
+        const float lprev = __uint_as_float(lprev_bits);   // sum of the E4M3 values
+        if (!SAGE) store_l(sLt, r, (j - 1) % kGroup, lprev);
+        ltot += lprev;
       }
       // tcgen05.ld/st are warp-collective: if any row of the warp rescales, the
       // whole warp runs the read-modify-write (other rows multiply by 1)
@@ -516,14 +555,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
           for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * rescale);
           VCA_TMEM_ST32(tO + c0, o);
         }
-        for (int kk = 0; kk < (SAGE ? 0 : j % kGroup); ++kk) {
+        // the L entries not yet restored: those of block j-1's group
+        for (int kk = 0; kk <= (SAGE ? -1 : (j - 1) % kGroup); ++kk) {
           float* hi = reinterpret_cast<float*>(sLt + tf32_tile_off(r, kk));
           float* lo = reinterpret_cast<float*>(sLt + 4096 + tf32_tile_off(r, kk));
           *hi *= rescale;
           *lo *= rescale;
         }
       }
-      ltot = ltot * rescale + l;
+      ltot *= rescale;
       // UE8M0 scale vectors for this PV: A = 2^0, B = 2^v_exp[j]
       {
         const uint32_t eb = (uint32_t)(127 + vex_j);
@@ -540,8 +580,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       tc_fence_before();
       mbar_arrive(&bars.p_full[t]);
     }
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ last row sums
+    // the last block's row sum completes the L tile (zero past the last block)
+    // and the total; the MMA warp then issues the last group's mean restore
     if (ok) ok = mbar_wait_warp(&bars.o_done[t], (nkv - 1) & 1, &abort_s, p.st, lim, 420 + t);
+    if (ok) {
+      tc_fence_after();
+      uint32_t lb = tmem_ld1(tRS);
+      tmem_ld_wait();
+      reg_after_wait(lb);
+      const float llast = __uint_as_float(lb);
+      ltot += llast;
+      if (!SAGE) {
+        const int kk = (nkv - 1) % kGroup;
+        store_l(sLt, r, kk, llast);
+        for (int k2 = kk + 1; k2 < kGroup; ++k2) store_l(sLt, r, k2, 0.0f);
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.p_full[t]);
+      ok = mbar_wait_warp(&bars.o_done[t], nkv & 1, &abort_s, p.st, lim, 430 + t);
+    }
+    // ------------------------------------------------------------ epilogue
     if (ok) {
       tc_fence_after();
       const int qrow = qtile * 128 + r;
