@@ -319,9 +319,10 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
         uint32_t c[2] = {0u, 0u};
         if (row < nv && m > 0.0f) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            c[q >> 1] |= (uint32_t)cvt_e4m3x2(__fmul_rn(bf16_lo(ws4[q]), inv), __fmul_rn(bf16_hi(ws4[q]), inv))
-                         << ((q & 1) * 16);
+          for (int q = 0; q < 4; ++q) {
+            const float2 y = __fmul2_rn(make_float2(bf16_lo(ws4[q]), bf16_hi(ws4[q])), make_float2(inv, inv));
+            c[q >> 1] |= (uint32_t)cvt_e4m3x2(y.x, y.y) << ((q & 1) * 16);
+          }
         }
         *reinterpret_cast<uint2*>(dst + (int64_t)row * 128 + chunk * 8) = make_uint2(c[0], c[1]);
       }
@@ -330,9 +331,14 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
       const int chunk = t & 15, g = t >> 4;
       uint4 w[8];
       uint32_t m2 = 0u;
-      int hs[8], ls[8];
+      // exact fixed-point sums: llrint(v 2^24) = hi 2^22 + lo per value (the
+      // split of fix24_split, two values per fma.rn.f32x2), summed as the raw
+      // bits magic + hi and magic + lo; the 8 magic constants of the 8 tokens
+      // are taken off once (wrap-around arithmetic, |sum| < 2^26)
+      uint32_t hs[8], ls[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) hs[c] = ls[c] = 0;
+      for (int c = 0; c < 8; ++c) hs[c] = ls[c] = 0u;
+      const float kMagic = 12582912.0f;   // 1.5 * 2^23
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int row = 8 * g + u;
@@ -342,14 +348,22 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
         const uint32_t ws4[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          int h, l;
-          fix24_split(bf16_lo(ws4[q]), h, l);
-          hs[2 * q] += h;
-          ls[2 * q] += l;
-          fix24_split(bf16_hi(ws4[q]), h, l);
-          hs[2 * q + 1] += h;
-          ls[2 * q + 1] += l;
+          const float2 v = make_float2(bf16_lo(ws4[q]), bf16_hi(ws4[q]));
+          // hm = magic + rne(4 v); r = v - hi / 4 (exact); lm = magic + rne(r 2^24)
+          const float2 hm = __ffma2_rn(v, make_float2(4.0f, 4.0f), make_float2(kMagic, kMagic));
+          const float2 hf = __fadd2_rn(hm, make_float2(-kMagic, -kMagic));
+          const float2 rr = __ffma2_rn(hf, make_float2(-0.25f, -0.25f), v);
+          const float2 lm = __ffma2_rn(rr, make_float2(16777216.0f, 16777216.0f), make_float2(kMagic, kMagic));
+          hs[2 * q] += __float_as_uint(hm.x);
+          hs[2 * q + 1] += __float_as_uint(hm.y);
+          ls[2 * q] += __float_as_uint(lm.x);
+          ls[2 * q + 1] += __float_as_uint(lm.y);
         }
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        hs[c] -= 8u * 0x4B400000u;
+        ls[c] -= 8u * 0x4B400000u;
       }
       // the tile is in registers: its stage now holds the partial sums and codes
       const bool anybad = compute_sync_or(max_half(m2) >= 0x4980u);   // |v| >= 2^20, inf or NaN
@@ -359,8 +373,8 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
       uint8_t* codeT = tile + 2 * 16 * 128 * 4;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        s_hi[g * 128 + 8 * chunk + c] = hs[c];
-        s_lo[g * 128 + 8 * chunk + c] = ls[c];
+        s_hi[g * 128 + 8 * chunk + c] = (int)hs[c];
+        s_lo[g * 128 + 8 * chunk + c] = (int)ls[c];
       }
       compute_sync();
       if (t < 128) {
@@ -371,7 +385,9 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
           L += s_lo[q * 128 + t];
         }
         const long long S = (long long)H * 4194304ll + (long long)L;
-        const uint16_t mb = double_to_bf16_rne(__ddiv_rn((double)S, (double)nv * 16777216.0));
+        // S / (nv 2^24): for a full block a division by 2^31, exact as a product
+        const double mean = nv == 128 ? (double)S * 0x1p-31 : __ddiv_rn((double)S, (double)nv * 16777216.0);
+        const uint16_t mb = double_to_bf16_rne(mean);
         a.v_mean[((int64_t)bh * nb + blk) * 128 + t] = mb;
         mu_s[t] = __uint_as_float((uint32_t)mb << 16);
       }
@@ -386,8 +402,9 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
           const uint32_t ws4[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            ramax = fmaxf(ramax, fabsf(__fsub_rn(bf16_lo(ws4[q]), mu[2 * q])));
-            ramax = fmaxf(ramax, fabsf(__fsub_rn(bf16_hi(ws4[q]), mu[2 * q + 1])));
+            const float2 y = __fadd2_rn(make_float2(bf16_lo(ws4[q]), bf16_hi(ws4[q])),
+                                        make_float2(-mu[2 * q], -mu[2 * q + 1]));
+            ramax = fmax3(ramax, fabsf(y.x), fabsf(y.y));
           }
         }
       }
@@ -395,15 +412,23 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
       const int e = v_exponent(m);
       if (t == 0) a.v_exp[(int64_t)bh * nb + blk] = (int8_t)e;
       const float sc = pow2_neg(e);
+      float musc[8];   // -mu * 2^-e (exact: a power of two times a bf16 value)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) musc[c] = -mu[c] * sc;
       uint32_t lo4[8], hi4[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const uint32_t ws4[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+        // (v - mu) * 2^-e, rounded once to fp32 by the subtraction; the power of
+        // two is applied exactly inside the same fma (fp32 results below 2^-126
+        // code to E4M3 zero either way)
         float x[8];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          x[2 * q] = __fmul_rn(__fsub_rn(bf16_lo(ws4[q]), mu[2 * q]), sc);
-          x[2 * q + 1] = __fmul_rn(__fsub_rn(bf16_hi(ws4[q]), mu[2 * q + 1]), sc);
+          const float2 y = __ffma2_rn(make_float2(bf16_lo(ws4[q]), bf16_hi(ws4[q])), make_float2(sc, sc),
+                                      make_float2(musc[2 * q], musc[2 * q + 1]));
+          x[2 * q] = y.x;
+          x[2 * q + 1] = y.y;
         }
         const bool valid = 8 * g + u < nv;
         lo4[u] = valid ? ((uint32_t)cvt_e4m3x2(x[0], x[1]) | ((uint32_t)cvt_e4m3x2(x[2], x[3]) << 16)) : 0u;
