@@ -195,11 +195,14 @@ __device__ __forceinline__ int compute_sync_or(int pred) {
                : "memory");
   return r;
 }
-__device__ __forceinline__ float compute_max(float v, float* red) {
+// Maximum of v over the 256 compute threads, and the OR of pred, with one
+// barrier.  red[] is rewritten here, so no thread may still be reading it
+// from an earlier call: every call is separated from the previous one by a
+// compute barrier (the per-item barrier at the top of the loop).
+__device__ __forceinline__ float compute_max_or(float v, int pred, float* red, int& any) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  compute_sync();
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-  compute_sync();
+  any = compute_sync_or(pred);
   float m = red[0];
   for (int i = 1; i < kPrepThreads / 32; ++i) m = fmaxf(m, red[i]);
   return m;
@@ -233,7 +236,6 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int N = a.N, nb = a.nb;
   const int64_t Np = (int64_t)nb * 128;
-  const long long items = 3ll * BH * nb;
   if (t == 0) {
     abort_s = 0;
     for (int i = 0; i < kStreamStages; ++i) {
@@ -243,24 +245,36 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
     fence_barrier_init();
   }
   __syncthreads();
-  // item -> (tensor, head, block): tensors interleaved so a CTA mixes all three
-  auto decode = [&](long long it, int& tensor, int& bh, int& blk) {
-    tensor = (int)(it % 3);
-    const long long rest = it / 3;
-    bh = (int)(rest / nb);
-    blk = (int)(rest % nb);
+  // Items it = blockIdx.x + k * gridDim.x, it = 3 (bh nb + blk) + tensor
+  // (tensors interleaved so a CTA mixes all three), walked by a cursor that
+  // adds the stride with carries: no 64-bit division per item.
+  struct Cursor {
+    int tensor, blk, bh;
   };
-  const long long first = blockIdx.x, step = gridDim.x;
+  const int step = gridDim.x;
+  const int st_t = step % 3, st_q = step / 3, st_b = st_q % nb, st_h = st_q / nb;
+  auto first_item = [&]() {
+    const int it = blockIdx.x, q = it / 3;
+    return Cursor{it % 3, q % nb, q / nb};
+  };
+  auto next_item = [&](Cursor& c) {
+    c.tensor += st_t;
+    const int c1 = c.tensor >= 3;
+    c.tensor -= 3 * c1;
+    c.blk += st_b + c1;
+    const int c2 = c.blk >= nb;
+    c.blk -= nb * c2;
+    c.bh += st_h + c2;
+  };
   if (warp == kPrepThreads / 32) {
     // ---- producer: item k goes to stage k % 3 once the compute warps released it
     int k = 0;
-    for (long long it = first; it < items; it += step, ++k) {
+    for (Cursor cur = first_item(); cur.bh < BH; next_item(cur), ++k) {
       const int stg = k % kStreamStages;
       if (k >= kStreamStages &&
           !mbar_wait_bounded(&empty[stg], ((k / kStreamStages) - 1) & 1, &abort_s, a.st, lim, 803))
         break;
-      int tensor, bh, blk;
-      decode(it, tensor, bh, blk);
+      const int tensor = cur.tensor, bh = cur.bh, blk = cur.blk;
       const int n0 = blk * 128, nv = min(128, N - n0);
       uint8_t* dst = stages + stg * kStageBytes;
       // the gathered rows' source indices first (one round trip), then the copies
@@ -286,13 +300,12 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
     return;
   }
   int k = 0;
-  for (long long it = first; it < items; it += step, ++k) {
+  for (Cursor cur = first_item(); cur.bh < BH; next_item(cur), ++k) {
     const int stg = k % kStreamStages;
     uint8_t* tile = stages + stg * kStageBytes;
     bool ok = mbar_wait_bounded(&full[stg], (k / kStreamStages) & 1, &abort_s, a.st, lim, 800);
     if (compute_sync_or(!ok)) break;
-    int tensor, bh, blk;
-    decode(it, tensor, bh, blk);
+    const int tensor = cur.tensor, bh = cur.bh, blk = cur.blk;
     const int n0 = blk * 128, nv = min(128, N - n0);
     if (tensor < 2) {
       // ---- Q / K: per-block fp32 scale, codes straight from registers
@@ -307,8 +320,9 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
         m2 = vmax_mag2(vmax_mag2(m2, w[i].z), w[i].w);
       }
       const uint32_t mbits = max_half(m2);
-      const float m = compute_max(__uint_as_float(mbits << 16), red);   // block max |x| (inf / NaN flagged)
-      if (compute_sync_or(mbits >= 0x7F80u) && t == 0) report(a.st, VCA_ERR_NONFINITE, 1 + tensor, blk);
+      int nonfinite;
+      const float m = compute_max_or(__uint_as_float(mbits << 16), mbits >= 0x7F80u, red, nonfinite);   // block max |x|
+      if (nonfinite && t == 0) report(a.st, VCA_ERR_NONFINITE, 1 + tensor, blk);
       const float inv = m > 0.0f ? __fdiv_rn(448.0f, m) : 0.0f;
       if (t == 0) (tensor == 0 ? a.q_scale : a.k_scale)[(int64_t)bh * nb + blk] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
       uint8_t* dst = (tensor == 0 ? a.Qq : a.Kq) + ((int64_t)bh * Np + n0) * 128;
@@ -408,7 +422,8 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
           }
         }
       }
-      const float m = compute_max(ramax, red);
+      int unused;
+      const float m = compute_max_or(ramax, 0, red, unused);
       const int e = v_exponent(m);
       if (t == 0) a.v_exp[(int64_t)bh * nb + blk] = (int8_t)e;
       const float sc = pow2_neg(e);
