@@ -26,7 +26,6 @@ namespace vca {
 
 constexpr int kPrepThreads = 256;
 constexpr int kTilePitch = 136;            // bf16 elements per smem row (pad 8)
-constexpr int kCodePitch = 144;            // bytes per smem row of the code tile
 
 struct PrepArgs {
   const uint16_t* Q;
@@ -171,9 +170,11 @@ __device__ __forceinline__ int vseg_swz(int c) { return 2 * ((c >> 3) & 7); }
 // ---------------------------------------------------------------- streaming form
 // vca_smooth_quantize_qkv's kernel: persistent CTAs walk the (block, tensor,
 // head) items; a producer warp (warp 8) fills a 3-stage ring of 32 KB token
-// tiles with bulk asynchronous copies (one copy for a block of Q, whose rows
-// are contiguous; one 256-byte copy per gathered row of K or V), so two blocks
-// stream in while the 8 compute warps code one.  The compute warps synchronise
+// tiles with 16-byte asynchronous copies (cp.async; for K and V each
+// instruction moves two whole gathered rows, lanes 0-15 and 16-31), so two
+// blocks stream in while the 8 compute warps code one.  (One bulk copy per
+// 256-byte gathered row kept the copy engine busy: the K and V tiles waited
+// ~4,000 cycles for their rows against ~120 for a Q tile in one bulk copy.)  The compute warps synchronise
 // among themselves on named barrier 1 and release a stage with one arrival
 // per warp.  The arithmetic per block is that of smooth_quant_kernel for Q
 // and K; the V scratch (exact partial sums and the
@@ -208,12 +209,17 @@ __device__ __forceinline__ float compute_max_or(float v, int pred, float* red, i
   return m;
 }
 
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
+// 16 bytes global -> shared (cp.async, cached in L2 only); completion is
+// reported through cp_async_mbar_arrive.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
+// Arrive on the barrier once every cp.async this thread issued before has
+// completed (.noinc: the arrival is one of the barrier's expected count).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 
 // Per 16-bit half, the larger of the two bf16 magnitude bit patterns (for
 // finite values these order like the magnitudes; inf and NaN are larger).
@@ -239,7 +245,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
   if (t == 0) {
     abort_s = 0;
     for (int i = 0; i < kStreamStages; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&full[i], 32);   // one arrival per producer lane
       mbar_init(&empty[i], kPrepThreads / 32);
     }
     fence_barrier_init();
@@ -277,25 +283,31 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
       const int tensor = cur.tensor, bh = cur.bh, blk = cur.blk;
       const int n0 = blk * 128, nv = min(128, N - n0);
       uint8_t* dst = stages + stg * kStageBytes;
-      // the gathered rows' source indices first (one round trip), then the copies
-      int src_row[4];
-      if (tensor != 0) {
+      if (tensor == 0) {
+        // Q rows are contiguous: lane l copies 16-byte chunks l, l + 32, ...
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(a.Q + ((int64_t)bh * N + n0) * 128);
+        for (int c = lane; c < nv * 16; c += 32) cp_async16(dst + c * 16, src + (int64_t)c * 16);
+      } else {
+        // gathered rows: the source indices first (one round trip), then per
+        // instruction two whole 256-byte rows (lanes 0-15 and 16-31)
         const int32_t* pm = a.perm + (int64_t)bh * N + n0;
+        int src_row[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) src_row[i] = lane + 32 * i < nv ? __ldg(pm + lane + 32 * i) : 0;
-      }
-      if (lane == 0) mbar_arrive_expect_tx(&full[stg], (uint32_t)nv * 256u);
-      __syncwarp();
-      if (tensor == 0) {
-        if (lane == 0) bulk_g2s(dst, a.Q + ((int64_t)bh * N + n0) * 128, (uint32_t)nv * 256u, &full[stg]);
-      } else {
-        const uint16_t* src = (tensor == 1 ? a.K : a.V) + (int64_t)bh * N * 128;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>((tensor == 1 ? a.K : a.V) + (int64_t)bh * N * 128);
+        const int half = lane >> 4, ch = lane & 15;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = lane + 32 * i;
-          if (r < nv) bulk_g2s(dst + r * 256, src + (int64_t)src_row[i] * 128, 256u, &full[stg]);
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int r = 32 * j + 2 * i + half;
+            const int srow = __shfl_sync(0xffffffffu, src_row[j], 2 * i + half);
+            if (r < nv) cp_async16(dst + r * 256 + ch * 16, src + (int64_t)srow * 256 + ch * 16);
+          }
         }
       }
+      // one arrival per lane, made once all of the lane's copies have landed
+      cp_async_mbar_arrive(&full[stg]);
     }
     return;
   }
