@@ -444,8 +444,9 @@ def run_ours(args, world, rank, local):
     line["fp4_prep"] = {"ms": round(fp4_ms, 3), "bound": "hbm", "algorithmic_bytes": fb,
                         "achieved": round(fb / (fp4_ms / 1e3) / 1e9, 1), "unit": "GB/s", "peak": peaks["hbm_gbs"],
                         "frac": round(fb / (fp4_ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
-                        "launches": 4, "what": "vca_smooth_quantize_qkv_fp4: Q/K E4M3 as the 8-bit prep, "
-                                              "V residual NVFP4 (two passes over V)"}
+                        "launches": 2, "what": "vca_smooth_quantize_qkv_fp4: one streaming launch for Q/K "
+                                              "(E4M3 as the 8-bit prep) and the first pass over V (means, head "
+                                              "maxima), one launch coding the NVFP4 V residual"}
     line["fp4_attention"] = {"ms": round(fp4_attn_ms, 3), "tflops": round(w.flops / (fp4_attn_ms / 1e3) / 1e12, 1),
                              "what": "vca_attention_fwd_fp4: QK^T E4M3, PV kind::mxf4nvf4 with NVFP4 probabilities "
                                      "(exp2 on the MUFU pipe) and NVFP4 V residual"}

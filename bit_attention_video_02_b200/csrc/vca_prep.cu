@@ -9,14 +9,15 @@
 //
 // vca_smooth_quantize_qkv runs one persistent kernel (smooth_quant_stream_kernel):
 // a producer warp streams 128-token tiles of Q, K and V (K and V rows gathered
-// through the permutation) into a 3-stage shared-memory ring with bulk
+// through the permutation) into a 3-stage shared-memory ring with 16-byte
 // asynchronous copies, and 8 compute warps code one tile while two more land.
 // Q/K tiles: per-block fp32 scale, codes written straight from registers.
 // V tiles: each thread holds 8 consecutive tokens x 8 channels; exact
 // per-channel sums and the residual maximum through shared-memory reductions;
 // the residual codes are transposed in registers so VrT rows (channel-major)
-// are written as full 128-byte lines.  smooth_quant_kernel (one CTA per Q or K
-// block) serves the 4-bit prep's Q and K.
+// are written as full 128-byte lines.  The 4-bit prep runs the same kernel for
+// Q, K and its first pass over V (block means, heads' residual maxima), then
+// smooth_quant_v4_kernel codes the NVFP4 residual.
 #include <algorithm>
 
 #include "vca_device.cuh"
@@ -41,7 +42,9 @@ struct PrepArgs {
   int8_t* v_exp;
   uint16_t* v_mean;
   DevStatus* st;
-  int tensor_base;   // blockIdx.y + tensor_base: 0 = Q, 1 = K, 2 = V
+  // 4-bit prep, first pass over V (streaming kernel): V blocks write their means
+  // and fold their residual maximum into head_amax[bh] instead of being coded
+  unsigned* head_amax;
 };
 
 // Smallest e with amax <= 448 * 2^e (0 for amax == 0), clamped to [-127, 127].
@@ -62,93 +65,6 @@ __device__ __forceinline__ float pow2_neg(int e) {
   if (k >= -126) return __uint_as_float((uint32_t)(k + 127) << 23);
   return __uint_as_float(0x00400000u);  // 2^-127
 }
-
-__device__ __forceinline__ float block_max(float v, float* red) {
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  int w = threadIdx.x >> 5;
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) red[w] = v;
-  __syncthreads();
-  float m = red[0];
-  for (int i = 1; i < kPrepThreads / 32; ++i) m = fmaxf(m, red[i]);
-  return m;
-}
-
-// The Q and K blocks: one CTA per (128-token block, tensor, head), tensor =
-// blockIdx.y + tensor_base (0 = Q, 1 = K).
-__global__ void __launch_bounds__(kPrepThreads) smooth_quant_kernel(const PrepArgs a) {
-  __shared__ float red[kPrepThreads / 32];
-  __shared__ int flag_s;
-
-  const int blk = blockIdx.x, tensor = blockIdx.y + a.tensor_base, bh = blockIdx.z;
-  const int N = a.N, nb = a.nb;
-  const int64_t Np = (int64_t)nb * 128;
-  const int n0 = blk * 128;
-  const int nv = min(128, N - n0);
-  const int t = threadIdx.x;
-  const int chunk = t & 15;          // 16-byte chunk (8 channels) of a row
-  const int rsub = t >> 4;           // 0..15
-
-  const uint16_t* src = tensor == 0 ? a.Q : a.K;
-  src += (int64_t)bh * N * 128;
-  const int32_t* perm = a.perm + (int64_t)bh * N;
-  if (t == 0) flag_s = 0;
-  __syncthreads();
-
-  // ---- load 128 rows x 128 channels (8 rows of 16 per thread pass)
-  uint4 w[8];
-  float amax = 0.0f;
-  int bad = 0;
-#pragma unroll
-  for (int it = 0; it < 8; ++it) {
-    int row = it * 16 + rsub;
-    w[it] = make_uint4(0, 0, 0, 0);
-    if (row < nv) {
-      int64_t srow = tensor == 0 ? (int64_t)(n0 + row) : (int64_t)__ldg(perm + n0 + row);
-      w[it] = __ldg(reinterpret_cast<const uint4*>(src + srow * 128) + chunk);
-      uint32_t ws4[4] = {w[it].x, w[it].y, w[it].z, w[it].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float lo = bf16_lo(ws4[q]), hi = bf16_hi(ws4[q]);
-        amax = fmaxf(amax, fmaxf(fabsf(lo), fabsf(hi)));
-        uint32_t elo = (ws4[q] >> 7) & 0xFFu, ehi = (ws4[q] >> 23) & 0xFFu;
-        bad |= (elo == 0xFF) | (ehi == 0xFF);
-      }
-    }
-  }
-  if (bad) flag_s = 1;
-
-  {
-    // ---- Q / K: per-block fp32 scale, codes straight from registers
-    float m = block_max(amax, red);
-    if (flag_s && t == 0) report(a.st, VCA_ERR_NONFINITE, 1 + tensor, blk);
-    float inv = 0.0f;
-    if (m > 0.0f) inv = __fdiv_rn(448.0f, m);
-    if (t == 0) {
-      float* sc = tensor == 0 ? a.q_scale : a.k_scale;
-      sc[(int64_t)bh * nb + blk] = m > 0.0f ? __fdiv_rn(m, 448.0f) : 1.0f;
-    }
-    uint8_t* dst = (tensor == 0 ? a.Qq : a.Kq) + ((int64_t)bh * Np + n0) * 128;
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      int row = it * 16 + rsub;
-      uint32_t ws4[4] = {w[it].x, w[it].y, w[it].z, w[it].w};
-      uint32_t c[2] = {0u, 0u};
-      if (row < nv && m > 0.0f) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t p = cvt_e4m3x2(__fmul_rn(bf16_lo(ws4[q]), inv), __fmul_rn(bf16_hi(ws4[q]), inv));
-          c[q >> 1] |= p << ((q & 1) * 16);
-        }
-      }
-      *reinterpret_cast<uint2*>(dst + (int64_t)row * 128 + chunk * 8) = make_uint2(c[0], c[1]);
-    }
-    return;
-  }
-
-}
-
-
 
 // 4 x 4 byte transpose: out[c] byte r = in[r] byte c.
 __device__ __forceinline__ void transpose4x4(const uint32_t in[4], uint32_t out[4]) {
@@ -176,9 +92,8 @@ __device__ __forceinline__ int vseg_swz(int c) { return 2 * ((c >> 3) & 7); }
 // 256-byte gathered row kept the copy engine busy: the K and V tiles waited
 // ~4,000 cycles for their rows against ~120 for a Q tile in one bulk copy.)  The compute warps synchronise
 // among themselves on named barrier 1 and release a stage with one arrival
-// per warp.  The arithmetic per block is that of smooth_quant_kernel for Q
-// and K; the V scratch (exact partial sums and the
-// code tile) reuses the stage of the block being coded.
+// per warp.  The V scratch (exact partial sums and the code tile) reuses the
+// stage of the block being coded.
 constexpr int kStreamStages = 3;
 constexpr uint32_t kStageBytes = 128 * 256;
 constexpr size_t kStreamSmem = kStreamStages * kStageBytes + 128;
@@ -436,6 +351,11 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
       }
       int unused;
       const float m = compute_max_or(ramax, 0, red, unused);
+      if (a.head_amax) {
+        // 4-bit prep, first pass: the head's residual maximum (fp32 bits of a
+        // non-negative value order like unsigned integers); coding comes later
+        if (t == 0) atomicMax(a.head_amax + bh, __float_as_uint(m));
+      } else {
       const int e = v_exponent(m);
       if (t == 0) a.v_exp[(int64_t)bh * nb + blk] = (int8_t)e;
       const float sc = pow2_neg(e);
@@ -486,6 +406,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2) smooth_quant_stream_kernel(
         const int c = idx >> 3, part = idx & 7;
         *reinterpret_cast<uint4*>(dstT + (int64_t)c * Np + 16 * (part ^ (vseg_swz(c) >> 1))) =
             *reinterpret_cast<const uint4*>(codeT + c * 128 + part * 16);
+      }
       }
     }
     // this warp is done with the stage (its reads and, for V, the scratch)
@@ -545,15 +466,13 @@ __device__ __forceinline__ uint32_t e2m1_code(float x) {
   return c | ((__float_as_uint(x) >> 31) << 3);
 }
 
-template <int PASS>
+// The 4-bit prep's second pass over V (the first ran in the streaming
+// kernel: block means in v_mean, the heads' residual maxima in head_amax).
 __global__ void __launch_bounds__(kPrepThreads) smooth_quant_v4_kernel(const PrepV4Args a) {
   extern __shared__ __align__(16) uint8_t sm[];
   uint16_t* tile = reinterpret_cast<uint16_t*>(sm);     // [128][136] bf16
-  uint8_t* codeT = sm + 128 * kTilePitch * 2;           // [128][80] u8 (second pass)
-  __shared__ float red[kPrepThreads / 32];
-  __shared__ long long psum[kPrepThreads];
+  uint8_t* codeT = sm + 128 * kTilePitch * 2;           // [128][80] u8
   __shared__ float mu_s[128];
-  __shared__ int flag_s;
 
   const int blk = blockIdx.x, bh = blockIdx.y;
   const int N = a.N, nb = a.nb;
@@ -564,58 +483,18 @@ __global__ void __launch_bounds__(kPrepThreads) smooth_quant_v4_kernel(const Pre
   const int chunk = t & 15, rsub = t >> 4;
   const uint16_t* src = a.V + (int64_t)bh * N * 128;
   const int32_t* perm = a.perm + (int64_t)bh * N;
-  if (t == 0) flag_s = 0;
-  __syncthreads();
 
   // ---- gather the block's 128 permuted value rows into shared memory
-  int bad = 0;
 #pragma unroll
   for (int it = 0; it < 8; ++it) {
     const int row = it * 16 + rsub;
     uint4 w = make_uint4(0, 0, 0, 0);
-    if (row < nv) {
-      w = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)__ldg(perm + n0 + row) * 128) + chunk);
-      if (PASS == 0) {
-        const uint32_t ws4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t elo = (ws4[q] >> 7) & 0xFFu, ehi = (ws4[q] >> 23) & 0xFFu;
-          bad |= (elo >= 147) | (ehi >= 147);   // non-finite or |v| >= 2^20
-        }
-      }
-    }
+    if (row < nv) w = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)__ldg(perm + n0 + row) * 128) + chunk);
     *reinterpret_cast<uint4*>(tile + row * kTilePitch + chunk * 8) = w;
   }
-  if (bad) flag_s = 1;
-  __syncthreads();
   const int ch = t & 127, half = t >> 7;
 
-  if (PASS == 0) {
-    if (flag_s && t == 0) report(a.st, VCA_ERR_NONFINITE, 3, blk);
-    // exact per-channel sums in 2^-24 fixed point (two threads per channel),
-    // one fp64 division, one rounding to bf16: the 8-bit prep's block mean
-    long long s = 0;
-    for (int r = half * 64; r < min(nv, half * 64 + 64); ++r)
-      s += __float2ll_rn(__uint_as_float((uint32_t)tile[r * kTilePitch + ch] << 16) * 16777216.0f);
-    psum[t] = s;
-    __syncthreads();
-    if (t < 128) {
-      const long long S = psum[t] + psum[t + 128];
-      const uint16_t mb = double_to_bf16_rne(__ddiv_rn((double)S, (double)nv * 16777216.0));
-      a.v_mean[((int64_t)bh * nb + blk) * 128 + t] = mb;
-      mu_s[t] = __uint_as_float((uint32_t)mb << 16);
-    }
-    __syncthreads();
-    const float mu = mu_s[ch];
-    float ramax = 0.0f;
-    for (int r = half * 64; r < min(nv, half * 64 + 64); ++r)
-      ramax = fmaxf(ramax, fabsf(__fsub_rn(__uint_as_float((uint32_t)tile[r * kTilePitch + ch] << 16), mu)));
-    const float m = block_max(ramax, red);
-    if (t == 0) atomicMax(a.head_amax + bh, __float_as_uint(m));
-    return;
-  }
-
-  // ---- second pass: code (channel, 16-token group) units, four per thread
+  // ---- code (channel, 16-token group) units, four per thread
   if (t < 128) mu_s[t] = __uint_as_float((uint32_t)a.v_mean[((int64_t)bh * nb + blk) * 128 + t] << 16);
   __syncthreads();
   const float hmax = __uint_as_float(a.head_amax[bh]);
@@ -664,8 +543,7 @@ __global__ void __launch_bounds__(kPrepThreads) smooth_quant_v4_kernel(const Pre
         *reinterpret_cast<const uint2*>(codeT + t * kV4Pitch + 64);
 }
 
-constexpr size_t kV4Smem0 = 128 * kTilePitch * 2;
-constexpr size_t kV4Smem1 = kV4Smem0 + 128 * kV4Pitch;
+constexpr size_t kV4Smem = 128 * kTilePitch * 2 + 128 * kV4Pitch;
 
 }  // namespace vca
 
@@ -699,7 +577,7 @@ extern "C" int vca_smooth_quantize_qkv(const vca_bf16* Q, const vca_bf16* K, con
   a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.N = N; a.nb = (N + 127) / 128;
   a.Qq = Qq; a.q_scale = q_scale; a.Kq = Kq; a.k_scale = k_scale; a.VrT = VrT;
   a.v_exp = v_exp; a.v_mean = v_mean; a.st = (DevStatus*)ws;
-  a.tensor_base = 0;
+  a.head_amax = nullptr;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = 3ll * B * H * a.nb;
@@ -732,23 +610,28 @@ extern "C" int vca_smooth_quantize_qkv_fp4(const vca_bf16* Q, const vca_bf16* K,
     return fail(VCA_ERR_WORKSPACE, "%s: workspace too small", fn);
   const int nb = (N + 127) / 128;
   cudaStream_t s = (cudaStream_t)stream;
-  // Q and K: the 8-bit prep's kernel, unchanged
+  unsigned* head_amax = reinterpret_cast<unsigned*>((char*)ws + 256);
+  if (cudaMemsetAsync(head_amax, 0, (size_t)B * H * 4, s) != cudaSuccess)
+    return fail(VCA_ERR_CUDA, "%s: memset failed", fn);
+  // Q, K (the 8-bit prep's codes) and the first pass over V (block means and
+  // the heads' residual maxima) in one persistent launch of the streaming kernel
+  if (cudaFuncSetAttribute(smooth_quant_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kStreamSmem) != cudaSuccess)
+    return fail(VCA_ERR_CUDA, "%s: cannot set shared-memory size", fn);
   PrepArgs a;
   a.Q = Q; a.K = K; a.V = V; a.perm = perm; a.N = N; a.nb = nb;
   a.Qq = Qq; a.q_scale = q_scale; a.Kq = Kq; a.k_scale = k_scale; a.VrT = nullptr;
-  a.v_exp = nullptr; a.v_mean = nullptr; a.st = (DevStatus*)ws; a.tensor_base = 0;
-  smooth_quant_kernel<<<dim3(nb, 2, B * H), kPrepThreads, 0, s>>>(a);
-  int rc = check_launch("smooth_quant_kernel (Q, K)");
+  a.v_exp = nullptr; a.v_mean = v_mean; a.st = (DevStatus*)ws; a.head_amax = head_amax;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = (int)std::min<long long>(3ll * B * H * nb, 2ll * sms);
+  smooth_quant_stream_kernel<<<grid, kStreamThreads, kStreamSmem, s>>>(a, B * H, wait_limit_ns());
+  int rc = check_launch("smooth_quant_stream_kernel (4-bit prep)");
   if (rc) return rc;
-  // V: block means and the head maxima, then the NVFP4 residual
+  // the NVFP4 residual, coded with the heads' tensor scales
   PrepV4Args v;
   v.V = V; v.perm = perm; v.N = N; v.nb = nb; v.VrT4 = VrT4; v.v_sc = v_sc; v.v_gscale = v_gscale;
-  v.v_mean = v_mean; v.head_amax = reinterpret_cast<unsigned*>((char*)ws + 256); v.st = (DevStatus*)ws;
-  if (cudaMemsetAsync(v.head_amax, 0, (size_t)B * H * 4, s) != cudaSuccess)
-    return fail(VCA_ERR_CUDA, "%s: memset failed", fn);
-  smooth_quant_v4_kernel<0><<<dim3(nb, B * H), kPrepThreads, kV4Smem0, s>>>(v);
-  rc = check_launch("smooth_quant_v4_kernel<0>");
-  if (rc) return rc;
-  smooth_quant_v4_kernel<1><<<dim3(nb, B * H), kPrepThreads, kV4Smem1, s>>>(v);
-  return check_launch("smooth_quant_v4_kernel<1>");
+  v.v_mean = v_mean; v.head_amax = head_amax; v.st = (DevStatus*)ws;
+  smooth_quant_v4_kernel<<<dim3(nb, B * H), kPrepThreads, kV4Smem, s>>>(v);
+  return check_launch("smooth_quant_v4_kernel");
 }
