@@ -161,16 +161,26 @@ __global__ void __launch_bounds__(kAssignThreads) km_assign_kernel(const uint16_
 
 // Exact fixed-point sums per (cluster, channel), walking the tokens in sorted
 // (cluster-contiguous) order.  Each warp takes kSegTok consecutive sorted
-// positions, lane l holding channels l + 32j.  llrint(v * 2^24) (|v| < 2^20, at
-// most 45 bits) is split exactly into hi * 2^22 + lo with |hi|, |lo| < 2^22 by
-// float operations only: f = v * 2^24 is exact, hi = trunc(f / 2^22),
-// lo = rne(f - hi * 2^22) (the only rounding, the same as llrint's), each made
-// an integer with the magic-number add.  The halves are summed in 32-bit
-// registers (at most kSegTok < 512 terms, so |sum| < 2^31) and flushed as one
-// int64 atomic per channel whenever the walk leaves a cluster.  Integer
-// addition is exact and order-free: the sums are exact whatever the order.
+// positions, lane l holding channels 4l .. 4l + 3 (a whole 256-byte row per
+// warp load, eight rows in flight).  llrint(v * 2^24) (|v| < 2^20, at most 45
+// bits) is split exactly into hi * 2^22 + lo with |hi| < 2^22, |lo| <= 2^21 by
+// float operations only: hi = rne(4 v) (exact product, one rounding through
+// the magic-number add), r = v - hi / 4 (exact), lo = rne(r * 2^24) (the only
+// other rounding, the same as llrint's since hi * 2^22 is an integer).  The
+// magic-biased bit patterns are summed in 32-bit registers and the bias is
+// taken off per token at each flush (at most kSegTok < 512 terms, so the true
+// sums stay below 2^31 and wrap-around is harmless); one int64 atomic per
+// channel is flushed whenever the walk leaves a cluster.  Integer addition is
+// exact and order-free: the sums are exact whatever the order.
 constexpr int kSegTok = 256;   // sorted positions per warp
 constexpr int kSegWarps = 8;
+// Per 16-bit half, the larger of two unsigned values.
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 __global__ void __launch_bounds__(kSegWarps * 32) km_accum_kernel(const uint16_t* __restrict__ V,
                                                                  const int32_t* __restrict__ perm,
                                                                  const int* __restrict__ cstart,
@@ -196,31 +206,38 @@ __global__ void __launch_bounds__(kSegWarps * 32) km_accum_kernel(const uint16_t
   const uint16_t* vb = V + (int64_t)bh * N * 128;
   const int32_t* pb = perm + (int64_t)bh * N;
   unsigned long long* sb = reinterpret_cast<unsigned long long*>(sums + (int64_t)bh * k * 128);
-  int hi[4] = {0, 0, 0, 0}, lo[4] = {0, 0, 0, 0};
-  uint32_t magbits = 0;   // largest |v| bit pattern seen: the exact sums need |v| < 2^20
+  // lane = channels 4 lane .. 4 lane + 3 (one 8-byte load per row); exact
+  // llrint(v 2^24) = hi 2^22 + lo per value, two values per fma.rn.f32x2, summed
+  // as the raw bits magic + hi / magic + lo and corrected by the token count at
+  // each flush (wrap-around arithmetic; |sum| < 2^31 over <= 256 tokens)
+  const float kMagic = 12582912.0f;   // 1.5 * 2^23
+  uint32_t hs[4] = {0u, 0u, 0u, 0u}, ls[4] = {0u, 0u, 0u, 0u};
+  uint32_t ntok = 0;
+  uint32_t mag2 = 0;   // largest |v| bit patterns seen (two halves): the exact sums need |v| < 2^20
   auto flush = [&]() {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const long long v = ((long long)hi[j] << 22) + (long long)lo[j];
-      if (v != 0) atomicAdd(sb + c * 128 + lane + 32 * j, (unsigned long long)v);
-      hi[j] = 0;
-      lo[j] = 0;
+      const int h = (int)(hs[j] - ntok * 0x4B400000u), l = (int)(ls[j] - ntok * 0x4B400000u);
+      const long long v = ((long long)h << 22) + (long long)l;
+      if (v != 0) atomicAdd(sb + c * 128 + 4 * lane + j, (unsigned long long)v);
+      hs[j] = 0u;
+      ls[j] = 0u;
     }
+    ntok = 0;
   };
   for (int base = q0; base < q1; base += 32) {
     const int cnt = min(32, q1 - base);
     const int myn = lane < cnt ? __ldg(pb + base + lane) : 0;
-    for (int i = 0; i < cnt; i += 4) {
-      // four tokens' rows in flight at once
-      uint16_t x[4][4];
+    for (int i = 0; i < cnt; i += 8) {
+      // eight tokens' rows in flight at once, each a 256-byte row per warp load
+      uint2 x[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const int n = __shfl_sync(0xffffffffu, myn, (i + u) & 31);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) x[u][j] = i + u < cnt ? __ldg(vb + (int64_t)n * 128 + lane + 32 * j) : (uint16_t)0;
+        x[u] = i + u < cnt ? __ldg(reinterpret_cast<const uint2*>(vb + (int64_t)n * 128) + lane) : make_uint2(0u, 0u);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         if (i + u >= cnt) break;
         const int q = base + i + u;
         if (q >= cend) {   // the walk enters the next non-empty cluster
@@ -230,20 +247,29 @@ __global__ void __launch_bounds__(kSegWarps * 32) km_accum_kernel(const uint16_t
           } while (c < k - 1 && ce[c] == cs[c]);
           cend = ce[c];
         }
+        mag2 = vmax_u16x2(mag2, x[u].x & 0x7FFF7FFFu);
+        mag2 = vmax_u16x2(mag2, x[u].y & 0x7FFF7FFFu);
+        const uint32_t wv[2] = {x[u].x, x[u].y};
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          int h, l;
-          magbits = max(magbits, (uint32_t)x[u][j] & 0x7FFFu);
-          fix24_split(__uint_as_float((uint32_t)x[u][j] << 16), h, l);
-          hi[j] += h;
-          lo[j] += l;
+        for (int p = 0; p < 2; ++p) {
+          const float2 v = make_float2(__uint_as_float(wv[p] << 16), __uint_as_float(wv[p] & 0xFFFF0000u));
+          // hm = magic + rne(4 v); r = v - hi / 4 (exact); lm = magic + rne(r 2^24)
+          const float2 hm = __ffma2_rn(v, make_float2(4.0f, 4.0f), make_float2(kMagic, kMagic));
+          const float2 hf = __fadd2_rn(hm, make_float2(-kMagic, -kMagic));
+          const float2 rr = __ffma2_rn(hf, make_float2(-0.25f, -0.25f), v);
+          const float2 lm = __ffma2_rn(rr, make_float2(16777216.0f, 16777216.0f), make_float2(kMagic, kMagic));
+          hs[2 * p] += __float_as_uint(hm.x);
+          hs[2 * p + 1] += __float_as_uint(hm.y);
+          ls[2 * p] += __float_as_uint(lm.x);
+          ls[2 * p + 1] += __float_as_uint(lm.y);
         }
+        ++ntok;
       }
     }
   }
   flush();
   // bf16 exponent field >= 127 + 20: |v| >= 2^20 (all ones: inf or NaN)
-  magbits = __reduce_max_sync(0xffffffffu, magbits);
+  const uint32_t magbits = __reduce_max_sync(0xffffffffu, max(mag2 & 0xFFFFu, mag2 >> 16));
   if (lane == 0 && magbits >= 0x4980u)
     report(st, magbits >= 0x7F80u ? VCA_ERR_NONFINITE : VCA_ERR_INVALID, 600, bh);
 }
