@@ -131,7 +131,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ int never_s;   // abort flag for drain waits: these must not give up early
-  __shared__ int warp_drop_s[2][4];   // Skip Softmax: warp w of tile t dropped the current block
+  // Skip Softmax: byte w of warp_drop_s[t] is 1 when warp w of tile t dropped the
+  // current block (one 32-bit read tells the MMA warp whether the whole tile did)
+  __shared__ uint32_t warp_drop_s[2];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x, bh = blockIdx.y;
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
   if (threadIdx.x == 0) {
     abort_s = 0;
     never_s = 0;
-    for (int i = 0; i < 8; ++i) warp_drop_s[i >> 2][i & 3] = 0;
+    warp_drop_s[0] = warp_drop_s[1] = 0u;
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars.kv_full[s], 1);
@@ -268,8 +270,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       // (the flags were written before the warpgroup's p_full arrivals)
       bool skip_pv = false;
       if (SKIP) {
-        const volatile int* f = warp_drop_s[t];
-        skip_pv = f[0] && f[1] && f[2] && f[3];
+        skip_pv = *reinterpret_cast<const volatile uint32_t*>(&warp_drop_s[t]) == 0x01010101u;
         nskip += skip_pv ? 1 : 0;
       }
       if (!SAGE && j > 0 && j % kGroup == 0 && !issue_mu(t, j / kGroup - 1)) return false;
@@ -574,7 +575,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         for (int i = 4; i < 8; ++i) sf[i] = eb * 0x01010101u;
         tmem_st8(tP, sf);
       }
-      if (SKIP && lane == 0) warp_drop_s[t][warp & 3] = warp_drop ? 1 : 0;
+      if (SKIP && lane == 0) reinterpret_cast<volatile uint8_t*>(&warp_drop_s[t])[warp & 3] = warp_drop ? 1 : 0;
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
