@@ -405,20 +405,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fp4_kernel(const __grid_cons
       uint32_t pw[16];   // 128 E2M1 codes, 8 per word, in key order
       uint32_t sfa[2];   // the 8 group scale codes, 4 per word
       float l = 0.0f;
+      const float2 czh2 = make_float2(cz_hi, cz_hi), czl2 = make_float2(cz_lo, cz_lo);
+      const float2 bias2 = make_float2(bias, bias);
 #pragma unroll
       for (int g = 0; g < 8; ++g) {
         float pv[16];
         float am = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < 16; i += 2) {
           // z - n - phi + 4 with z = s (cz_hi + cz_lo): the product's rounding
-          // error recovered by an fma, the small terms added last
-          const float s_ = sv[16 * g + i];
-          const float zh = s_ * cz_hi;
-          const float zl = __fmaf_rn(s_, cz_lo, __fmaf_rn(s_, cz_hi, -zh));
-          pv[i] = ex2_approx((zh + bias) + zl);
-          if (valid < 128 && 16 * g + i >= valid) pv[i] = 0.0f;   // keys past the end (the error term is NaN there)
-          am = fmaxf(am, pv[i]);
+          // error recovered by an fma, the small terms added last (two scores
+          // per f32x2 instruction, each element rounded as the scalar form)
+          const float2 s2 = make_float2(sv[16 * g + i], sv[16 * g + i + 1]);
+          const float2 zh = __fmul2_rn(s2, czh2);
+          const float2 zl = __ffma2_rn(s2, czl2, __ffma2_rn(s2, czh2, make_float2(-zh.x, -zh.y)));
+          const float2 a = __fadd2_rn(__fadd2_rn(zh, bias2), zl);
+          pv[i] = ex2_approx(a.x);
+          pv[i + 1] = ex2_approx(a.y);
+          if (valid < 128) {   // keys past the end (the error term is NaN there)
+            if (16 * g + i >= valid) pv[i] = 0.0f;
+            if (16 * g + i + 1 >= valid) pv[i + 1] = 0.0f;
+          }
+          am = fmax3(am, pv[i], pv[i + 1]);
         }
         const uint32_t sc = cvt_e4m3x2(__fdiv_rn(am, 0.75f), 0.0f) & 0xFFu;
         const float s = __uint_as_float(sc << 20) * 0x1p120f;   // decode(sc), exact
@@ -429,7 +437,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fp4_kernel(const __grid_cons
           const float inv = __frcp_rn(sg);
           uint32_t b[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) b[i] = cvt_e2m1x2(__fmul_rn(pv[2 * i], inv), __fmul_rn(pv[2 * i + 1], inv));
+          for (int i = 0; i < 8; ++i) {
+            const float2 y = __fmul2_rn(make_float2(pv[2 * i], pv[2 * i + 1]), make_float2(inv, inv));
+            b[i] = cvt_e2m1x2(y.x, y.y);
+          }
           w0 = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
           w1 = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
           __half2 acc = __halves2half2(__float2half_rn(0.0f), __float2half_rn(0.0f));
