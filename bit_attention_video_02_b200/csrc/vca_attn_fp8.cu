@@ -15,8 +15,9 @@
 //    means, warps 4-7 / 8-11 are the softmax warpgroups of query tile 0 / 1
 //    (thread = query row = TMEM lane).
 //  * TMEM (512 columns): S (one fp32 score tile, shared by the two query
-//    tiles in turn), the P region (per tile: two 4-column UE8M0 scale vectors
-//    and 32 columns of packed E4M3 codes), O0, O1 (fp32 accumulators).
+//    tiles in turn), O0, O1 (fp32 accumulators of 144 columns: the 128 output
+//    channels and the block row sum), per tile 32 columns of packed E4M3 codes,
+//    and the UE8M0 scale vectors (A's shared, B's double-buffered by key block).
 //  * S = Q_t K_j^T: tcgen05 kind::f8f6f4, operands from 128B-swizzled smem.
 //    A softmax warpgroup releases S as soon as it has loaded its scores into
 //    registers, and the MMA warp refills it for the other tile, so the tensor
@@ -26,7 +27,10 @@
 //      QK0(0) QK1(0) QK0(1) | PV0(j) QK1(j+1) PV1(j) QK0(j+2) | ...
 //  * O_t += P_t R_j * 2^e_j: kind::mxf8f6f4.block_scale with A = P_t read
 //    from tensor memory (no shared-memory round trip for the probabilities);
-//    the per-block V exponent is the UE8M0 scale of B (A's scale is 1).  A
+//    the per-block V exponent is the UE8M0 scale of B (A's scale is 1).  B has
+//    144 rows: the V tile and a constant row of E4M3 ones (scale 2^0), so the
+//    same MMAs leave the block row sum of the decoded codes in column 128 of
+//    O_t, which the warpgroup reads and zeroes while coding the next block.  A
 //    warpgroup writes P_t(j) and the scale vectors only after PV_t(j-1) has
 //    completed (o_done), which it needs anyway before rescaling O_t.
 //  * Mean restore: every 8 key blocks, O_t += L_t M^T with a TF32 MMA, where
@@ -52,19 +56,24 @@ constexpr int kGroup = 8;   // key blocks per mean-restore MMA
 
 // TMEM columns
 constexpr uint32_t kColS = 0;     // score tile (128 columns)
-constexpr uint32_t kColP = 128;   // P region: tile t at +64t: scale vectors +0..+7, codes +8..+39,
-                                  // block row sum (16-column MMA output, column 0 used) +48..+63
-constexpr uint32_t kColRowSum = 48;
-constexpr uint32_t kColO = 256;   // O_t at +128t
+// O_t: 144 columns, the 128 output channels and (column 128) the block row sum
+// that PV accumulates against a ones row of B; the rest holds the P codes and
+// the UE8M0 scale vectors (A's shared by both tiles: all 2^0; B's double-
+// buffered by key-block parity: 2^e_j for the 128 channels, 2^0 for the ones rows)
+constexpr uint32_t kColO0 = 128, kColO1 = 288;
+constexpr uint32_t kColSFA = 272;
+constexpr uint32_t kColSFB0 = 276, kColSFB1 = 496;
+constexpr uint32_t kColCodes0 = 432, kColCodes1 = 464;
+constexpr int kPvN = 144;
 
 // dynamic shared memory layout (offsets from a 1024-aligned base)
 constexpr uint32_t kOffQ = 0;                         // 2 x 16 KB
 constexpr uint32_t kOffK = 32768;                     // kStages x 16 KB
-constexpr uint32_t kOffV = kOffK + kStages * 16384;   // kStages x 16 KB
-constexpr uint32_t kOffL = kOffV + kStages * 16384;   // 2 tiles x (hi 4 KB + lo 4 KB)
+constexpr uint32_t kVStage = 18432;                   // a V tile (16 KB) + 16 constant rows (2 KB)
+constexpr uint32_t kOffV = kOffK + kStages * 16384;   // kStages x 18 KB
+constexpr uint32_t kOffL = kOffV + kStages * kVStage; // 2 tiles x (hi 4 KB + lo 4 KB)
 constexpr uint32_t kOffMu = kOffL + 16384;            // 2 buffers x 4 KB
-constexpr uint32_t kOffOnes = kOffMu + 8192;          // 16 x 32 E4M3: row 0 ones, rows 1-15 zero
-constexpr uint32_t kSmemBytes = kOffOnes + 1024;
+constexpr uint32_t kSmemBytes = kOffMu + 8192;
 constexpr uint32_t kSmemAlloc = kSmemBytes + 1024;
 
 struct AttnParams {
@@ -115,6 +124,15 @@ __device__ __forceinline__ uint32_t tf32_tile_off(int r, int k) {
 // applied to the output and no block exponents or means (no mean restore).
 // QI8 (SAGE only): Q and K are INT8 codes, QK^T runs as kind::i8 into s32
 // accumulators, converted exactly to fp32 (|q.k| < 2^21) after the load.
+// one / four 32-bit TMEM columns of this thread's lane <- registers
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v));
+}
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3]));
+}
+
 // block row sum l -> L tile entry (row r, block kk of the group): the hi part
 // exact in TF32, lo the remainder
 __device__ __forceinline__ void store_l(uint8_t* sLt, int r, int kk, float l) {
@@ -165,16 +183,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     tma_prefetch_desc(&p.tmK);
     tma_prefetch_desc(&p.tmV);
   }
-  // the row-sum operand: B [16 x 32] K-major, no swizzle (core matrices of 8
-  // rows x 16 bytes, 128 bytes apart along K, 256 apart along N); row 0 holds
-  // E4M3 1.0 (0x38), rows 1-15 zero.  Every K step of the row-sum MMA reads it.
-  if (threadIdx.x < 128) {
-    const int off = threadIdx.x * 4;   // 512 bytes
-    const int in_cm = off & 127;       // byte within a core matrix: row (in_cm / 16)
-    const bool row0 = (off < 256) && (in_cm < 16);
-    *reinterpret_cast<uint32_t*>(sm + kOffOnes + off) = row0 ? 0x38383838u : 0u;
-    fence_proxy_async_smem();
+  // rows 128-143 of every V stage (after the 16 KB the TMA fills): row 128 all
+  // E4M3 1.0, the rest zero, so PV's B operand has a row of ones and its
+  // column 128 of O accumulates the row sum (the 128-byte swizzle permutes 16-byte
+  // chunks within a row, which leaves a constant row as it is)
+  for (int i = threadIdx.x; i < kStages * 512; i += kAttnThreads) {
+    const int s = i >> 9, off = (i & 511) * 4;
+    *reinterpret_cast<uint32_t*>(sm + kOffV + s * kVStage + 16384 + off) = off < 128 ? 0x38383838u : 0u;
   }
+  fence_proxy_async_smem();
   // a CTA of this launch (or of an earlier one sharing the workspace) already
   // timed out: do no work, so a broken pipeline costs one wait, not one per CTA
   __shared__ int skip_s;
@@ -203,7 +220,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         if (u > 0 && !mbar_wait_bounded(&bars.kv_empty[s], (u - 1) & 1, &abort_s, p.st, lim, 100)) break;
         mbar_arrive_expect_tx(&bars.kv_full[s], 32768);
         tma_load_2d(sm + kOffK + s * 16384, &p.tmK, &bars.kv_full[s], 0, (int)((int64_t)bh * Np) + j * 128);
-        tma_load_2d(sm + kOffV + s * 16384, &p.tmV, &bars.kv_full[s], j * 128, bh * 128);
+        tma_load_2d(sm + kOffV + s * kVStage, &p.tmV, &bars.kv_full[s], j * 128, bh * 128);
         issued = j + 1;
       }
       if (abort_s) {
@@ -220,10 +237,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     // with two softmax warps: the fewer instructions per MMA, the sooner the
     // tensor pipe gets its next operation.)
     const uint32_t id_qk = QI8 ? instr_desc_s8(128, 128) : instr_desc(kFmtE4M3, kFmtE4M3, 128, 128, 0, 0);
-    const uint32_t id_pv = instr_desc_mx(kFmtE4M3, kFmtE4M3, 128, 128);
+    const uint32_t id_pv = instr_desc_mx(kFmtE4M3, kFmtE4M3, 128, kPvN);
     const uint32_t id_mu = instr_desc(kFmtTF32, kFmtTF32, 128, 128, 0, 0);
-    const uint32_t id_rs = instr_desc(kFmtE4M3, kFmtE4M3, 128, 16, 0, 0);
-    const uint64_t dOnes = smem_desc(smem_u32(sm + kOffOnes), 128, 256, kLayoutNone);
     // descriptor start addresses count 16-byte units: +2 per 32-byte K step,
     // +1024 per 16 KB tile, +256 per 4 KB
     const uint64_t dQ = smem_desc(smem_u32(sm + kOffQ), 16, 1024, kLayoutSW128);
@@ -252,21 +267,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       if (!mbar_wait_warp(&bars.mu_full[gb], (g >> 1) & 1, &abort_s, p.st, lim, 220)) return false;
       tc_fence_after();
       const uint64_t bdesc = dMu + (uint64_t)(gb * 256);
-      mma_tf32_ss_w(tmem + kColO + t * 128, dL + (uint64_t)(t * 512), bdesc, id_mu, 1u);
-      mma_tf32_ss_w(tmem + kColO + t * 128, dL + (uint64_t)(t * 512 + 256), bdesc, id_mu, 1u);
+      const uint32_t tOt = tmem + (t ? kColO1 : kColO0);
+      mma_tf32_ss_w(tOt, dL + (uint64_t)(t * 512), bdesc, id_mu, 1u);
+      mma_tf32_ss_w(tOt, dL + (uint64_t)(t * 512 + 256), bdesc, id_mu, 1u);
       if (t == 1) tc_commit_w(&bars.mu_empty[gb]);
       return true;
     };
-    // O_t += P_t(j) R_j 2^e_j and the block row sums P_t(j) 1 (into the P
-    // region); the L tile of a group is complete once the warpgroup has read
+    // O_t += P_t(j) R_j 2^e_j, and in column 128 the block row sum P_t(j) 1 (B's
+    // ones row); the L tile of a group is complete once the warpgroup has read
     // the row sums of its last block, so a group's mean restore is issued with
     // the next group's first PV (the last group's after the loop).  o_done[t]
-    // then tracks everything that reads the P region or writes O_t.
+    // then tracks everything that reads P_t or the scale vectors, or writes O_t.
     auto issue_pv = [&](int t, int j) -> bool {
       if (!mbar_wait_warp(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t)) return false;
       tc_fence_after();
       const int s = j % kStages;
-      const uint32_t tP = tmem + kColP + t * 64;   // scale vectors at +0 / +4, codes at +8..+39
+      const uint32_t tCodes = tmem + (t ? kColCodes1 : kColCodes0);
+      const uint32_t tSFB = tmem + ((j & 1) ? kColSFB1 : kColSFB0);
       // (the flags were written before the warpgroup's p_full arrivals)
       bool skip_pv = false;
       if (SKIP) {
@@ -277,12 +294,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       if (!skip_pv) {
 #pragma unroll
         for (int k = 0; k < 4; ++k)   // 8 columns (32 codes) per K step
-          mma_mxf8_ts_w(tmem + kColO + t * 128, tP + 8 + 8 * k, dV + (uint64_t)(s * 1024 + 2 * k), id_pv, tP,
-                        tP + 4, (j > 0 || k > 0) ? 1u : 0u);
+          mma_mxf8_ts_w(tmem + (t ? kColO1 : kColO0), tCodes + 8 * k, dV + (uint64_t)(s * (kVStage / 16) + 2 * k),
+                        id_pv, tmem + kColSFA, tSFB, (j > 0 || k > 0) ? 1u : 0u);
       }
-#pragma unroll
-      for (int k = 0; k < 4; ++k)   // row sums: the same codes against a column of ones
-        mma_f8_ts_w(tP + kColRowSum, tP + 8 + 8 * k, dOnes, id_rs, k > 0 ? 1u : 0u);
       tc_commit_w(&bars.o_done[t]);
       return true;
     };
@@ -363,9 +377,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     const int r = threadIdx.x & 127;               // query row within the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + kColS + lane_off;
-    const uint32_t tP = tmem + kColP + t * 64 + lane_off;   // scale vectors +0..+7, codes +8..+39
-    const uint32_t tO = tmem + kColO + t * 128 + lane_off;
-    const uint32_t tRS = tP + kColRowSum;          // this row's block row sum (column 0)
+    const uint32_t tCodes = tmem + (t ? kColCodes1 : kColCodes0) + lane_off;   // this tile's P codes
+    const uint32_t tO = tmem + (t ? kColO1 : kColO0) + lane_off;
+    const uint32_t tRS = tO + 128;                 // the row sum PV accumulates (read and zeroed per block)
     const int qtile = pair * 2 + t;
     const bool qvalid = qtile < nb;
     const bool row_valid = qvalid && qtile * 128 + r < N;
@@ -496,8 +510,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       }
       // ExpCast: code = rne(s*c8 + 87 - 8*nref) via the magic-number FMA (two
       // scores per fma.rn.f32x2), clamped below at 0; the block's row sum of the
-      // decoded probabilities comes from the tensor core (the codes against a
-      // column of ones), read one block later
+      // decoded probabilities comes from the tensor core (PV's row of ones, in
+      // column 128 of O_t), read one block later
       const bool warp_drop = SKIP && __all_sync(0xffffffffu, rej);
       // a dropped row writes code 0 everywhere: multiplier 0, addend the bare magic constant
       const float badd = rej ? kMagic : kMagic + (float)(87 - 8 * nref);
@@ -519,7 +533,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       if (warp_drop) {
         // PV may still run for the other warps' rows: these rows contribute zeros
         const uint32_t zero[32] = {};
-        VCA_TMEM_ST32(tP + 8, zero);
+        VCA_TMEM_ST32(tCodes, zero);
       } else {
 #pragma unroll
       for (int q = 0; q < 32; ++q) {
@@ -532,13 +546,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         const uint32_t b2 = __float_as_uint(fmaxf(f23.x, kMagic)), b3 = __float_as_uint(fmaxf(f23.y, kMagic));
         pw[q] = prmt(prmt(b0, b1, 0x0040u), prmt(b2, b3, 0x0040u), 0x5410u);
       }
-      VCA_TMEM_ST32(tP + 8, pw);
+      VCA_TMEM_ST32(tCodes, pw);
       }
       if (j > 0) {
         // block j-1's row sum (in the units of the reference before this
         // block's rescale) -> L tile and the running total
         tmem_ld_wait();
         reg_after_wait(lprev_bits);
+        tmem_st1(tRS, 0u);   // the next PV adds block j's row sum to zero
         const float lprev = __uint_as_float(lprev_bits);   // sum of the E4M3 values
         if (!SAGE) store_l(sLt, r, (j - 1) % kGroup, lprev);
         ltot += lprev;
@@ -565,15 +580,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         }
       }
       ltot *= rescale;
-      // UE8M0 scale vectors for this PV: A = 2^0, B = 2^v_exp[j]
-      {
-        const uint32_t eb = (uint32_t)(127 + vex_j);
-        uint32_t sf[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sf[i] = 0x7F7F7F7Fu;
-#pragma unroll
-        for (int i = 4; i < 8; ++i) sf[i] = eb * 0x01010101u;
-        tmem_st8(tP, sf);
+      // UE8M0 scale vectors, written by tile 0's warpgroup (the PV of tile 1 for
+      // the same key block comes after tile 0's): A = 2^0 (once), B = 2^v_exp[j]
+      // for the 128 channel rows and 2^0 for the ones rows (fifth column)
+      if (t == 0) {
+        if (j == 0) {
+          const uint32_t one4[4] = {0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu};
+          tmem_st4(tmem + kColSFA + lane_off, one4);
+        }
+        const uint32_t eb = (uint32_t)(127 + vex_j) * 0x01010101u;
+        const uint32_t sf[8] = {eb, eb, eb, eb, 0x7F7F7F7Fu, 0u, 0u, 0u};
+        tmem_st8(tmem + ((j & 1) ? kColSFB1 : kColSFB0) + lane_off, sf);
       }
       if (SKIP && lane == 0) reinterpret_cast<volatile uint8_t*>(&warp_drop_s[t])[warp & 3] = warp_drop ? 1 : 0;
       fence_proxy_async_smem();
