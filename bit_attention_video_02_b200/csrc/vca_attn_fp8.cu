@@ -124,6 +124,24 @@ __device__ __forceinline__ uint32_t tf32_tile_off(int r, int k) {
 // applied to the output and no block exponents or means (no mean restore).
 // QI8 (SAGE only): Q and K are INT8 codes, QK^T runs as kind::i8 into s32
 // accumulators, converted exactly to fp32 (|q.k| < 2^21) after the load.
+// 64 consecutive 32-bit TMEM columns of this thread's lane -> registers.
+#define VCA_TMEM_LD64(taddr, r)                                                                     \
+  asm volatile(                                                                                     \
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15," \
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38," \
+      "%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61," \
+      "%62,%63}, [%64];"                                                                            \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), \
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),        \
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),      \
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),      \
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]),      \
+        "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]),      \
+        "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),      \
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]),      \
+        "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])       \
+      : "r"(taddr))
+
 // one / four 32-bit TMEM columns of this thread's lane <- registers
 __device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v));
@@ -430,10 +448,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
       float sv[128];
       {
         uint32_t* su = reinterpret_cast<uint32_t*>(sv);
-        VCA_TMEM_LD32(tS + 0, (su + 0));
-        VCA_TMEM_LD32(tS + 32, (su + 32));
-        VCA_TMEM_LD32(tS + 64, (su + 64));
-        VCA_TMEM_LD32(tS + 96, (su + 96));
+        VCA_TMEM_LD64(tS + 0, (su + 0));
+        VCA_TMEM_LD64(tS + 64, (su + 64));
         tmem_ld_wait();
       }
       // the scores are in registers: S may take the other tile's next scores
