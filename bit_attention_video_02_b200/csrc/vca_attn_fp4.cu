@@ -226,10 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fp4_kernel(const __grid_cons
     const uint32_t tS = tmem + kColS;
     auto issue_qk = [&](int t, int jj) {
       const int s1 = jj % kStages;
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        mma_f8_ss_w(tS, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(s1 * 1024 + 2 * k), id_qk, k > 0);
-      tc_commit_w(&bars.s_full[t]);
+      VCA_MMA4_SS_W("f8f6f4", tS, dQ + (uint64_t)(t * 1024), dK + (uint64_t)(s1 * 1024), id_qk, 0u, &bars.s_full[t]);
     };
     auto issue_pv = [&](int t, int j) -> bool {
       if (!mbar_wait_warp(&bars.p_full[t], j & 1, &abort_s, p.st, lim, 210 + t)) return false;

@@ -251,9 +251,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs this loop in lockstep, so descriptors are computed
     // once, stay warp-uniform and advance by constants; one elected lane issues
-    // each tcgen05 instruction.  (The issuing warp shares its SM sub-partition
-    // with two softmax warps: the fewer instructions per MMA, the sooner the
-    // tensor pipe gets its next operation.)
+    // the tcgen05 instructions, one election per QK^T or PV (its four K steps
+    // and the commit).  (The issuing warp shares its SM sub-partition with two
+    // softmax warps: the fewer instructions per MMA, the sooner the tensor pipe
+    // gets its next operation.)
     const uint32_t id_qk = QI8 ? instr_desc_s8(128, 128) : instr_desc(kFmtE4M3, kFmtE4M3, 128, 128, 0, 0);
     const uint32_t id_pv = instr_desc_mx(kFmtE4M3, kFmtE4M3, 128, kPvN);
     const uint32_t id_mu = instr_desc(kFmtTF32, kFmtTF32, 128, 128, 0, 0);
@@ -269,14 +270,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
     // S <- Q_t K_jj^T (K_jj in stage jj % kStages, already waited for)
     auto issue_qk = [&](int t, int jj) {
       const int s1 = jj % kStages;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (QI8)
-          mma_i8_ss_w(tS, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(s1 * 1024 + 2 * k), id_qk, k > 0);
-        else
-          mma_f8_ss_w(tS, dQ + (uint64_t)(t * 1024 + 2 * k), dK + (uint64_t)(s1 * 1024 + 2 * k), id_qk, k > 0);
-      }
-      tc_commit_w(&bars.s_full[t]);
+      if (QI8)
+        VCA_MMA4_SS_W("i8", tS, dQ + (uint64_t)(t * 1024), dK + (uint64_t)(s1 * 1024), id_qk, 0u, &bars.s_full[t]);
+      else
+        VCA_MMA4_SS_W("f8f6f4", tS, dQ + (uint64_t)(t * 1024), dK + (uint64_t)(s1 * 1024), id_qk, 0u,
+                      &bars.s_full[t]);
     };
     // mean restore of group g: O_t += L_t(g) M(g) (L split hi + lo); after
     // tile 1's, the block-mean buffer may be refilled
@@ -309,13 +307,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fp8_kernel(const __grid_
         nskip += skip_pv ? 1 : 0;
       }
       if (!SAGE && j > 0 && j % kGroup == 0 && !issue_mu(t, j / kGroup - 1)) return false;
-      if (!skip_pv) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k)   // 8 columns (32 codes) per K step
-          mma_mxf8_ts_w(tmem + (t ? kColO1 : kColO0), tCodes + 8 * k, dV + (uint64_t)(s * (kVStage / 16) + 2 * k),
-                        id_pv, tmem + kColSFA, tSFB, (j > 0 || k > 0) ? 1u : 0u);
-      }
-      tc_commit_w(&bars.o_done[t]);
+      if (!skip_pv)   // 8 columns (32 codes) per K step
+        VCA_MMA4_MXF8_TS_W(tmem + (t ? kColO1 : kColO0), tCodes, dV + (uint64_t)(s * (kVStage / 16)), id_pv,
+                           tmem + kColSFA, tSFB, j > 0 ? 1u : 0u, &bars.o_done[t]);
+      else
+        tc_commit_w(&bars.o_done[t]);
       return true;
     };
     // after the last block: the warpgroup has added the last row sums to the

@@ -150,35 +150,6 @@ __device__ __forceinline__ void tc_fence_after() {
 // instructions) and elect.sync picks the issuing lane -- lane 0 whenever all 32
 // lanes are active, so MMAs and the commits that track them come from the same
 // thread.
-__device__ __forceinline__ void mma_f8_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                            uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum));
-}
-__device__ __forceinline__ void mma_f8_ts_w(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                            uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accum));
-}
-__device__ __forceinline__ void mma_i8_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
-                                            uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accum));
-}
-__device__ __forceinline__ void mma_mxf8_ts_w(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
-                                              uint32_t sfa, uint32_t sfb, uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %6, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], [%1], %2, %3, [%4], [%5], p;\n\t}" ::"r"(
-          d),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accum));
-}
 __device__ __forceinline__ void mma_tf32_ss_w(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
                                               uint32_t accum) {
   asm volatile(
@@ -207,6 +178,43 @@ __device__ __forceinline__ void tc_commit_w(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
+
+// The four 32-byte K steps of a K = 128 contraction of 8-bit operands and the
+// commit that follows them, issued by one lane that a single elect.sync picks
+// (one elect per group instead of one per instruction).  Step k reads the
+// shared-memory descriptors advanced by 2k (16-byte units) and, for an A operand
+// in tensor memory, the columns advanced by 8k; the first step accumulates iff
+// accum0 != 0, the others always.  KIND is the tcgen05.mma kind as a string
+// literal ("f8f6f4", "i8").
+#define VCA_MMA4_SS_W(KIND, d, a, b, idesc, accum0, bar)                                            \
+  asm volatile("{\n\t.reg .pred e, p0, p1;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"               \
+               "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"                 \
+               "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"                 \
+               "setp.ne.b32 p0, %4, 0;\n\tsetp.eq.b32 p1, %4, %4;\n\t"                              \
+               "elect.sync _|e, 0xffffffff;\n\t"                                                    \
+               "@e tcgen05.mma.cta_group::1.kind::" KIND " [%0], %1, %2, %3, p0;\n\t"             \
+               "@e tcgen05.mma.cta_group::1.kind::" KIND " [%0], a1, b1, %3, p1;\n\t"             \
+               "@e tcgen05.mma.cta_group::1.kind::" KIND " [%0], a2, b2, %3, p1;\n\t"             \
+               "@e tcgen05.mma.cta_group::1.kind::" KIND " [%0], a3, b3, %3, p1;\n\t"             \
+               "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t}" \
+               ::"r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accum0), "r"(smem_u32(bar))                \
+               : "memory")
+// The same for the block-scaled E4M3 x E4M3 MMA with A (the P codes) in tensor
+// memory and the UE8M0 scale vectors at sfa / sfb.
+#define VCA_MMA4_MXF8_TS_W(d, a_tmem, b, idesc, sfa, sfb, accum0, bar)                               \
+  asm volatile("{\n\t.reg .pred e, p0, p1;\n\t.reg .b64 b1, b2, b3;\n\t.reg .b32 a1, a2, a3;\n\t"   \
+               "add.s32 a1, %1, 8;\n\tadd.s32 a2, %1, 16;\n\tadd.s32 a3, %1, 24;\n\t"               \
+               "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"                 \
+               "setp.ne.b32 p0, %6, 0;\n\tsetp.eq.b32 p1, %6, %6;\n\t"                              \
+               "elect.sync _|e, 0xffffffff;\n\t"                                                    \
+               "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], [%1], %2, %3, [%4], [%5], p0;\n\t" \
+               "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], [a1], b1, %3, [%4], [%5], p1;\n\t" \
+               "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], [a2], b2, %3, [%4], [%5], p1;\n\t" \
+               "@e tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], [a3], b3, %3, [%4], [%5], p1;\n\t" \
+               "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t}" \
+               ::"r"(d), "r"(a_tmem), "l"(b), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accum0),           \
+                 "r"(smem_u32(bar))                                                                 \
+               : "memory")
 
 // 32 consecutive 32-bit TMEM columns of this thread's lane -> registers.
 #define VCA_TMEM_LD32(taddr, r)                                                                  \

@@ -453,9 +453,6 @@ extern "C" int vca_cluster_permute(const vca_bf16* V, int B, int H, int N, int d
 
 static __device__ __align__(256) unsigned char g_cluster_scratch[VCA_NOALLOC_SCRATCH_BYTES];
 
-// The array's host-side name is only a stand-in for the symbol; the device
-// address comes from cudaGetSymbolAddress, looked up once per device with that
-// device current (the first call on each device does it).
 // The array's device address, looked up on every call (the lookup allocates
 // nothing, and after a device reset the address may differ) with the
 // caller's device current.
