@@ -6,6 +6,9 @@
 // and attention are all per head), so the layer is cut into chunks of heads and
 // run as a three-stage pipeline over two device slots: copy chunk c+1 in while
 // chunk c is grouped, quantised and attended, and copy chunk c-1's output out.
+// A slot's Q, K and V are dead once the quantiser has read them, so the next
+// input copy into that slot waits only for that, and the attention that
+// rewrites its O waits for the output copy.
 // Each chunk runs exactly the per-head kernels of vca_cluster_permute,
 // vca_smooth_quantize_qkv and vca_attention_fwd, so the result is the same, bit
 // for bit, as running the three calls on the whole layer.
@@ -81,31 +84,50 @@ int get_streams(Streams* out) {
   return VCA_OK;
 }
 
-// Chunk boundaries: sizes double from one unit up to `u` (1, 2, 4, ..., u, u, ...)
-// and the last chunk holds one unit.  The first chunk's input copy and the last
-// chunk's output copy are the only transfers nothing overlaps, so they are kept
-// small; doubling lets each chunk's input copy fit under the previous chunk's
-// compute while the pipeline fills.  starts[i] is the first unit of chunk i,
+// Chunk boundaries.  A chunk of s units takes about 0.8 s units' compute time to
+// copy in while the output copy runs the other way (B200 over PCIe: ≈ 1.3 ms per
+// Wan-shaped head in, ≈ 1.7 ms of kernels), so the sizes grow by 1.5x from one
+// unit up to `u`: each chunk's input copy then fits under the previous chunk's
+// compute while the pipeline fills.  The last two chunks hold 3 units and 1
+// unit, so the output copy that nothing overlaps is one unit's and the one
+// before it fits under that unit's compute.  The units between are split
+// evenly into chunks of at most u.  starts[i] is the first unit of chunk i,
 // starts.back() == units.
 std::vector<int> chunk_starts(int units, int u) {
+  std::vector<int> head, tail, sizes;
+  int used = 0;
+  for (int s = 1; s < u && used + s <= units; s = (3 * s + 1) / 2 < u ? (3 * s + 1) / 2 : u) {
+    head.push_back(s);
+    used += s;
+  }
+  for (int t : {1, 3}) {
+    const int s = t < u ? t : u;
+    if (used + s > units) break;
+    tail.push_back(s);
+    used += s;
+  }
+  const int rest = units - used;
+  sizes = head;
+  if (rest > 0) {
+    const int nm = (rest + u - 1) / u, base = rest / nm, extra = rest % nm;
+    for (int i = 0; i < nm; ++i) sizes.push_back(base + (i < extra ? 1 : 0));
+  }
+  sizes.insert(sizes.end(), tail.rbegin(), tail.rend());
   std::vector<int> starts;
-  int pos = 0, size = 1;
-  while (pos < units) {
-    const int remaining = units - pos;
-    int take = size < remaining ? size : remaining;
-    if (take == remaining && remaining > 1) take = remaining - 1;   // the last unit goes alone
+  int pos = 0;
+  for (int s : sizes) {
     starts.push_back(pos);
-    pos += take;
-    size = 2 * size < u ? 2 * size : u;
+    pos += s;
   }
   starts.push_back(units);
   return starts;
 }
 
-// The seven events of one call (start, and per slot: input landed, compute
-// done, output copied), destroyed on every return path.
+// The nine events of one call (start, and per slot: input landed, input read
+// by the quantiser, compute done, output copied), destroyed on every return
+// path.
 struct Events {
-  cudaEvent_t e[7] = {};
+  cudaEvent_t e[9] = {};
   bool create() {
     for (cudaEvent_t& x : e)
       if (cudaEventCreateWithFlags(&x, cudaEventDisableTiming) != cudaSuccess) return false;
@@ -119,7 +141,7 @@ struct Events {
 
 int units_per_chunk(int units, int heads_per_chunk) {
   if (heads_per_chunk > 0) return heads_per_chunk < units ? heads_per_chunk : units;
-  const int u = (units + 4) / 5;   // about five chunks at full size, after the doubling ramp
+  const int u = (units + 3) / 4;   // about four chunks at full size, between the ramps
   return u < 1 ? 1 : u;
 }
 
@@ -151,7 +173,7 @@ extern "C" int vca_vc_attention_host(const vca_bf16* Q, const vca_bf16* K, const
   // the pipeline starts after the work already queued on the caller's stream
   Events evs;
   if (!evs.create()) return fail(VCA_ERR_CUDA, "%s: cannot create events", fn);
-  cudaEvent_t start = evs.e[0], *ev_in = evs.e + 1, *ev_done = evs.e + 3, *ev_free = evs.e + 5;
+  cudaEvent_t start = evs.e[0], *ev_in = evs.e + 1, *ev_read = evs.e + 3, *ev_done = evs.e + 5, *ev_free = evs.e + 7;
   cudaEventRecord(start, (cudaStream_t)stream);
   cudaStreamWaitEvent(st.h2d, start, 0);
   cudaStreamWaitEvent(st.comp, start, 0);
@@ -168,8 +190,10 @@ extern "C" int vca_vc_attention_host(const vca_bf16* Q, const vca_bf16* K, const
     const int u0 = starts[c], uc = starts[c + 1] - u0;
     char* b = base + (size_t)s * L.total;
     const size_t bytes = (size_t)uc * row * 2;
-    // slot s is free once chunk c-2's output has left the device
-    if (c >= 2) cudaStreamWaitEvent(st.h2d, ev_free[s], 0);
+    // slot s takes new inputs once chunk c-2's quantiser has read its Q, K, V
+    // (attention reads only the codes), and a new output once chunk c-2's O
+    // has left the device (below)
+    if (c >= 2) cudaStreamWaitEvent(st.h2d, ev_read[s], 0);
     if (cudaMemcpyAsync(b + L.q, Q + (size_t)u0 * row, bytes, cudaMemcpyHostToDevice, st.h2d) != cudaSuccess ||
         cudaMemcpyAsync(b + L.k, K + (size_t)u0 * row, bytes, cudaMemcpyHostToDevice, st.h2d) != cudaSuccess ||
         cudaMemcpyAsync(b + L.v, V + (size_t)u0 * row, bytes, cudaMemcpyHostToDevice, st.h2d) != cudaSuccess) {
@@ -188,10 +212,13 @@ extern "C" int vca_vc_attention_host(const vca_bf16* Q, const vca_bf16* K, const
                                    N, d, 128, (uint8_t*)(b + L.qq), (float*)(b + L.qs), (uint8_t*)(b + L.kq),
                                    (float*)(b + L.ks), (uint8_t*)(b + L.vrt), (int8_t*)(b + L.ve),
                                    (vca_bf16*)(b + L.vm), ws, wsb, st.comp);
-    if (!rc)
+    if (!rc) {
+      cudaEventRecord(ev_read[s], st.comp);
+      if (c >= 2) cudaStreamWaitEvent(st.comp, ev_free[s], 0);
       rc = vca_attention_fwd((uint8_t*)(b + L.qq), (float*)(b + L.qs), (uint8_t*)(b + L.kq), (float*)(b + L.ks),
                              (uint8_t*)(b + L.vrt), (int8_t*)(b + L.ve), (vca_bf16*)(b + L.vm), 1, uc, N, d,
                              softmax_scale, (vca_bf16*)(b + L.o), nullptr, ws, wsb, st.comp);
+    }
     if (rc) break;
     cudaEventRecord(ev_done[s], st.comp);
     cudaStreamWaitEvent(st.d2h, ev_done[s], 0);

@@ -304,12 +304,14 @@ int vca_attention_fwd_skip(const uint8_t* Qq, const float* q_scale, const uint8_
  * vca_attention_fwd), with the copies overlapped with the kernels.  The pages
  * have no counterpart: it serves callers whose activations live in host memory.
  * (b, h) units are independent, so the layer runs in chunks of
- * up to `heads_per_chunk` units (0 = a fifth of the layer) through a three-stage
- * pipeline on library-owned streams over two device slots: copy chunk c+1 in,
- * compute chunk c, copy chunk c-1 out.  Chunk sizes double from one unit up to
- * heads_per_chunk and the last chunk is one unit, so the transfers nothing
- * overlaps stay small.  Results equal the three calls on the whole layer bit
- * for bit.
+ * up to `heads_per_chunk` units (0 = a quarter of the layer) through a
+ * three-stage pipeline on library-owned streams over two device slots: copy
+ * chunk c+1 in, compute chunk c, copy chunk c-1 out.  A slot takes its next
+ * inputs as soon as the quantiser has read the previous ones, and its next
+ * output once the previous one has been copied out.  Chunk sizes grow by 1.5x
+ * from one unit up to heads_per_chunk and the last two chunks hold 3 units and
+ * 1, so the transfers nothing overlaps stay small.  Results equal the three
+ * calls on the whole layer bit for bit.
  *   Q, K, V   [B][H][N][d] bf16, HOST memory (in); page-locked memory
  *             (cudaHostAlloc / cudaHostRegister) is needed for the copies to
  *             overlap -- pageable memory works but serialises them

@@ -27,6 +27,18 @@ def test_host_pipeline_equals_device_path(heads_per_chunk):
     assert torch.equal(O, ref)
 
 
+@pytest.mark.parametrize("heads_per_chunk", [0, 4])
+def test_host_pipeline_ramp_and_tail(heads_per_chunk):
+    # 13 heads: chunks of 1, 2, 3 (ramp), the middle, then 3 and 1 (tail); the
+    # slots are reused while the previous chunk's attention or output copy runs
+    w = W.shrink(W.WORKLOADS[2], H=13, N=900)
+    Q, K, V = W.make_qkv(w, "cuda")
+    ref = _device_path(Q, K, V, w.k, 3).cpu()
+    hQ, hK, hV = (t.cpu().pin_memory() for t in (Q, K, V))
+    for _ in range(2):
+        assert torch.equal(vca.vc_attention_host(hQ, hK, hV, k=w.k, iters=3, heads_per_chunk=heads_per_chunk), ref)
+
+
 def test_host_pipeline_pageable_memory_and_repeat_calls():
     w = W.shrink(W.WORKLOADS[1], H=2, N=700)
     Q, K, V = W.make_qkv(w, "cuda")
