@@ -10,7 +10,9 @@
 // sorting.
 //
 // Per round: assign (token-parallel; fp32 distances in channel order, one FMA
-// per channel, so the argmin is reproducible bit for bit), accumulate
+// per channel, so the argmin is reproducible bit for bit; a tensor-core
+// estimate with a proven error bound picks the centroids whose distance is
+// evaluated), accumulate
 // (channel-parallel exact 2^-24 fixed-point sums in int64, order-free), update
 // (one fp64 division per centroid coordinate).  Then a stable counting sort:
 // per-chunk histograms, an exclusive scan in (cluster, chunk) order, and a
@@ -22,7 +24,6 @@
 
 namespace vca {
 
-constexpr int kAssignThreads = 128;
 constexpr int kSortChunk = 1024;    // tokens per sort CTA
 
 struct KmWs {
@@ -70,93 +71,225 @@ __global__ void km_init_kernel(const uint16_t* __restrict__ V, const float* __re
   }
 }
 
-// Shared-memory centroid table for the assignment: pairs of centroids
-// interleaved per channel and negated, cs[p][ch] = (-mu_{2p}[ch], -mu_{2p+1}[ch]),
-// so one fma.rn.f32x2 advances the distances to two centroids.  An odd k is
-// padded with a centroid at infinity, which never wins.  The channel loop is
-// outside the centroid loop, so each bf16 channel is unpacked once per token
-// and feeds NP accumulator pairs; every accumulator still adds its channels
-// in order 0..127 (the distance's defined summation order).
-template <int NP>
-__global__ void __launch_bounds__(kAssignThreads) km_assign_kernel(const uint16_t* __restrict__ V,
-                                                                  const float* __restrict__ cent,
-                                                                  int32_t* __restrict__ assign,
-                                                                  int N, int k) {
-  extern __shared__ float4 cs4[];   // [NP][64] float4 = [pairs][128 channels][2]
-  const int bh = blockIdx.y;
-  const int npairs = (k + 1) >> 1;
-  const float* src = cent + (int64_t)bh * k * 128;
-  float2* cs2 = reinterpret_cast<float2*>(cs4);
-  for (int i = threadIdx.x; i < NP * 128; i += blockDim.x) {
-    const int pp = i >> 7, ch = i & 127, c0 = 2 * pp, c1 = 2 * pp + 1;
-    cs2[i] = make_float2(c0 < k ? -src[c0 * 128 + ch] : -INFINITY, c1 < k ? -src[c1 * 128 + ch] : -INFINITY);
+// ---------------------------------------------------------------- assignment
+// The assignment keeps the distance's defined arithmetic -- for centroid mu,
+// t_i = v_i - mu_i rounded to fp32 and D = fma(t_i, t_i, D) over the channels
+// in order 0..127 from D = 0, the lowest index winning ties -- but evaluates it
+// only for the centroids that can win.  A tensor-core estimate
+//   d_c = |v|^2 + |mu_c|^2 - 2 v.mu_c
+// (v.mu_c from the bf16 V tile against the centroids split into bf16 hi + lo,
+// both accumulated in fp32 in tensor memory) differs from the defined D_c by less
+// than e_c = 2^-10 (|v|^2 + |mu_c|^2) + 2^-90:
+//  * the split leaves at most 2^-18 |mu_i| per coordinate, the bf16 products
+//    are exact, and the fp32 sums of at most 256 products err by less than
+//    2^-14 of their absolute sum, which is at most (|v|^2 + |mu|^2) / 2;
+//  * |v|^2 and |mu|^2 are fp32 sums of 128 exact squares (error below 2^-17
+//    of each), and the last two operations round once each;
+//  * D_c itself is within 131 units of 2^-24 of the exact squared distance,
+//    which is at most 2 (|v|^2 + |mu|^2);
+// together below 10^-4 of |v|^2 + |mu_c|^2, a tenth of the margin, and the
+// absolute term covers subnormal flushing.  Every centroid whose D_c is the
+// minimum therefore satisfies d_c - e_c <= min_k (d_k + e_k); the exact D is
+// computed for those candidates only, in increasing index, which gives the
+// full scan's result bit for bit.  A non-finite estimate anywhere sends the
+// token through all k centroids in the defined way.
+constexpr int kAsgThreads = 128;              // one token per thread = TMEM lane
+constexpr float kFilterRel = 0x1p-10f, kFilterAbs = 0x1p-90f;
+
+struct AsgParams {
+  CUtensorMap tmV;     // V as [BH][N][128] bf16; box 64 channels x 128 tokens, 128-byte swizzle
+  const float* cent;   // [BH][k][128]
+  int32_t* assign;     // [BH][N]
+  DevStatus* st;
+  uint64_t lim;
+  int N, k;
+};
+
+// KP centroid slots (32 for k <= 32, else 64): two B matrices of KP rows, the
+// bf16 hi parts and the lo parts of the centroids, accumulated into the same
+// KP tensor-memory columns (column c = v.hi_c + v.lo_c, 256 products).
+template <int KP>
+__global__ void __launch_bounds__(kAsgThreads, 4) km_assign_kernel(const __grid_constant__ AsgParams p) {
+  constexpr uint32_t kBChunk = KP * 128;   // bytes of one 64-channel chunk of a B matrix
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint8_t* sV = sm;           // the token tile: 2 chunks of 64 channels x 128 rows of 128 bytes
+  uint8_t* sB = sm + 32768;   // hi then lo, each 2 chunks of KP rows
+  __shared__ __align__(8) uint64_t bar_full, bar_mma;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s, never_s;
+  __shared__ float nc_s[KP];
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int bh = blockIdx.y, tile = blockIdx.x, k = p.k;
+  if (tid == 0) {
+    abort_s = 0;
+    never_s = 0;
+    mbar_init(&bar_full, 1);
+    mbar_init(&bar_mma, 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(&bar_full, 32768);
+    tma_load_3d(sV, &p.tmV, &bar_full, 0, tile * 128, bh);
+    tma_load_3d(sV + 16384, &p.tmV, &bar_full, 64, tile * 128, bh);
   }
+  // B: thread pair (c, half) writes centroid c's channels 64 half .. +63 as bf16
+  // hi and lo (row c of either matrix) in 16-byte units swizzled by the row
+  // index (the layout of a 128-byte-swizzle TMA box) and sums |mu_c|^2
+  {
+    const int c = tid >> 1, half = tid & 1;
+    if (c < KP) {   // warp-uniform: a warp holds 16 consecutive c
+      const float4* src = reinterpret_cast<const float4*>(p.cent + ((int64_t)bh * k + (c < k ? c : 0)) * 128) +
+                          half * 16;
+      uint8_t* hrow = sB + half * kBChunk + c * 128;
+      uint8_t* lrow = sB + (2 + half) * kBChunk + c * 128;
+      float ss = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {   // channels 64 half + 8u .. +7
+        float4 a = make_float4(0.0f, 0.0f, 0.0f, 0.0f), b = a;
+        if (c < k) {
+          a = __ldg(src + 2 * u);
+          b = __ldg(src + 2 * u + 1);
+        }
+        const float m[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(m[2 * e]), h1 = __float2bfloat16_rn(m[2 * e + 1]);
+          const __nv_bfloat16 l0 = __float2bfloat16_rn(m[2 * e] - __bfloat162float(h0));
+          const __nv_bfloat16 l1 = __float2bfloat16_rn(m[2 * e + 1] - __bfloat162float(h1));
+          hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+          lw[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+          ss = fmaf(m[2 * e], m[2 * e], ss);
+          ss = fmaf(m[2 * e + 1], m[2 * e + 1], ss);
+        }
+        const int su = (u ^ (c & 7)) << 4;
+        *reinterpret_cast<uint4*>(hrow + su) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(lrow + su) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+      if (half == 0) nc_s[c] = ss;
+    }
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_base_s, KP);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();   // B's rows, written by these threads, for the tensor core
+  tc_fence_before();
   __syncthreads();
-  // two tokens per thread (n and n + blockDim.x): every centroid value read from
-  // shared memory serves both
-  const int n = blockIdx.x * 2 * blockDim.x + threadIdx.x, nb2 = n + blockDim.x;
-  if (n >= N) return;
-  const bool has_b = nb2 < N;
-  const uint4* row = reinterpret_cast<const uint4*>(V + ((int64_t)bh * N + n) * 128);
-  const uint4* rowb = reinterpret_cast<const uint4*>(V + ((int64_t)bh * N + (has_b ? nb2 : n)) * 128);
-  float2 acc[NP], accb[NP];
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  bool issued = false;
+  if (warp == 0) {
+    // D[token][c] = sum over the 128 channels of v (hi_c + lo_c): 8 steps of 16
+    // channels against each matrix
+    issued = mbar_wait_warp(&bar_full, 0, &abort_s, p.st, p.lim, 500);
+    if (issued) {
+      tc_fence_after();
+      const uint32_t idesc = instr_desc(kFmtBF16, kFmtBF16, 128, KP, 0, 0);
+      const uint64_t dA = smem_desc(smem_u32(sV), 16, 1024, kLayoutSW128);
+      const uint64_t dB = smem_desc(smem_u32(sB), 16, 1024, kLayoutSW128);
 #pragma unroll
-  for (int pp = 0; pp < NP; ++pp) acc[pp] = accb[pp] = make_float2(0.0f, 0.0f);
-  // 8 channels per step; the next 16-byte pieces of the rows are loaded one step ahead
-  uint4 cur = __ldg(row), curb = __ldg(rowb);
-#pragma unroll 1
-  for (int q = 0; q < 16; ++q) {
-    const int qn = q + 1 < 16 ? q + 1 : q;
-    const uint4 nxt = __ldg(row + qn), nxtb = __ldg(rowb + qn);
-    const uint32_t w[4] = {cur.x, cur.y, cur.z, cur.w}, wb[4] = {curb.x, curb.y, curb.z, curb.w};
+      for (int s = 0; s < 16; ++s) {   // +32 bytes per step inside a 128-byte row, then the next chunk
+        const int st = s & 7;
+        mma_bf16_ss_w(tmem, dA + (uint64_t)((st >> 2) * 1024 + (st & 3) * 2),
+                      dB + (uint64_t)(((s >> 3) * 2 + (st >> 2)) * (kBChunk / 16) + (st & 3) * 2), idesc, s > 0);
+      }
+      tc_commit_w(&bar_mma);
+    }
+  }
+  // this thread's token: row tid of the tile (16-byte units swizzled by the
+  // row index), and |v|^2
+  bool ok = mbar_wait_warp(&bar_full, 0, &abort_s, p.st, p.lim, 501);
+  const uint8_t* vrow = sV + tid * 128;
+  const int vsw = tid & 7;
+  float nv = 0.0f;
+  if (ok) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = 4 * q + u;   // channels 2i, 2i+1
-      const float x0 = __uint_as_float(w[u] << 16), x1 = __uint_as_float(w[u] & 0xFFFF0000u);
-      const float y0 = __uint_as_float(wb[u] << 16), y1 = __uint_as_float(wb[u] & 0xFFFF0000u);
-      const float2 X0 = make_float2(x0, x0), X1 = make_float2(x1, x1);
-      const float2 Y0 = make_float2(y0, y0), Y1 = make_float2(y1, y1);
+    for (int u = 0; u < 16; ++u) {
+      const uint4 x = *reinterpret_cast<const uint4*>(vrow + (u >> 3) * 16384 + (((u & 7) ^ vsw) << 4));
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-      for (int pp = 0; pp < NP; ++pp) {
-        const float4 m = cs4[pp * 64 + i];   // channels 2i (x, y) and 2i+1 (z, w)
-        const float2 m0 = make_float2(m.x, m.y), m1 = make_float2(m.z, m.w);
-        float2 t = __fadd2_rn(X0, m0);   // v - mu, exact order per lane
-        acc[pp] = __ffma2_rn(t, t, acc[pp]);
-        t = __fadd2_rn(X1, m1);
-        acc[pp] = __ffma2_rn(t, t, acc[pp]);
-        t = __fadd2_rn(Y0, m0);
-        accb[pp] = __ffma2_rn(t, t, accb[pp]);
-        t = __fadd2_rn(Y1, m1);
-        accb[pp] = __ffma2_rn(t, t, accb[pp]);
+      for (int e = 0; e < 4; ++e) {
+        nv = fmaf(bf16_lo(w[e]), bf16_lo(w[e]), nv);
+        nv = fmaf(bf16_hi(w[e]), bf16_hi(w[e]), nv);
       }
     }
-    cur = nxt;
-    curb = nxtb;
   }
-  int best = 0, bestb = 0;
-  float bd = acc[0].x, bdb = accb[0].x;
+  ok = ok && mbar_wait_warp(&bar_mma, 0, &abort_s, p.st, p.lim, 502);
+  if (ok) {
+    tc_fence_after();
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    // pass 1: the smallest upper bound; pass 2: the candidates
+    float best_ub = INFINITY;
+    bool bad = !(fabsf(nv) < INFINITY);
+    uint64_t cand = 0;
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll 1
+      for (int g = 0; g < KP / 32; ++g) {
+        uint32_t dv[32];
+        VCA_TMEM_LD32(trow + 32 * g, dv);
+        tmem_ld_wait();
 #pragma unroll
-  for (int pp = 0; pp < NP; ++pp) {
-    if (pp > 0 && acc[pp].x < bd) {
-      bd = acc[pp].x;
-      best = 2 * pp;
+        for (int j = 0; j < 32; ++j) {
+          const int c = 32 * g + j;
+          if (c < k) {
+            const float dot = __uint_as_float(dv[j]);
+            const float sn = nv + nc_s[c];
+            const float d = fmaf(-2.0f, dot, sn);
+            const float e = fmaf(kFilterRel, sn, kFilterAbs);
+            if (pass == 0) {
+              best_ub = fminf(best_ub, d + e);
+              bad = bad || !(fabsf(d) < INFINITY);
+            } else if (d - e <= best_ub) {
+              cand |= 1ull << c;
+            }
+          }
+        }
+      }
     }
-    if (acc[pp].y < bd) {
-      bd = acc[pp].y;
-      best = 2 * pp + 1;
+    if (bad || !(best_ub < INFINITY)) cand = k == 64 ? ~0ull : (1ull << k) - 1;
+    // the defined distance for the candidates, in increasing index
+    const float4* cb = reinterpret_cast<const float4*>(p.cent + (int64_t)bh * k * 128);
+    int best = 0;
+    float bd = 0.0f;
+    bool first = true;
+    while (cand) {
+      const int c = __ffsll((long long)cand) - 1;
+      cand &= cand - 1;
+      const float4* mu = cb + c * 32;
+      float acc = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {   // channels 8u .. 8u + 7
+        const uint4 x = *reinterpret_cast<const uint4*>(vrow + (u >> 3) * 16384 + (((u & 7) ^ vsw) << 4));
+        const float4 m0 = __ldg(mu + 2 * u), m1 = __ldg(mu + 2 * u + 1);
+        const float vv[8] = {bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y),
+                             bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w)};
+        const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float t = __fsub_rn(vv[e], mm[e]);
+          acc = __fmaf_rn(t, t, acc);
+        }
+      }
+      if (first || acc < bd) {
+        bd = acc;
+        best = c;
+        first = false;
+      }
     }
-    if (pp > 0 && accb[pp].x < bdb) {
-      bdb = accb[pp].x;
-      bestb = 2 * pp;
-    }
-    if (accb[pp].y < bdb) {
-      bdb = accb[pp].y;
-      bestb = 2 * pp + 1;
-    }
+    const int n = tile * 128 + tid;
+    if (n < p.N) p.assign[(int64_t)bh * p.N + n] = best;
   }
-  if (has_b) assign[(int64_t)bh * N + nb2] = bestb;
-  (void)npairs;
-  assign[(int64_t)bh * N + n] = best;
+  // nothing may be in flight into this CTA's memory when it exits
+  if (tid == 0 && !ok) mbar_wait_bounded(&bar_full, 0, &never_s, nullptr, p.lim, 503);
+  if (warp == 0 && issued && !ok) mbar_wait_warp(&bar_mma, 0, &never_s, nullptr, p.lim, 504);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, KP);
+  }
 }
 
 // Exact fixed-point sums per (cluster, channel), walking the tokens in sorted
@@ -381,21 +514,35 @@ static int cluster_permute_impl(const vca_bf16* V, int B, int H, int N, int d, i
   km_init_kernel<<<dim3(BH, k), 128, 0, s>>>(V, init, cent, N, k);
   int rc = check_launch("km_init_kernel");
   if (rc) return rc;
-  // centroid table padded to 16 or 32 pairs (pads sit at infinity)
-  const int np = (k + 1) / 2 <= 16 ? 16 : 32;
-  const size_t assign_smem = (size_t)np * 128 * sizeof(float2);
-  auto assign_kernel = np == 16 ? km_assign_kernel<16> : km_assign_kernel<32>;
+  // the assignment's V tiles by TMA: [BH][N][128] bf16, 64 channels x 128 tokens
+  // per box, so tokens past N read as zero and are not written
+  AsgParams ap;
+  {
+    const uint64_t dims[3] = {128, (uint64_t)N, (uint64_t)BH}, str[2] = {256, (uint64_t)N * 256};
+    const uint32_t box[3] = {64, 128, 1};
+    rc = encode_tiled(&ap.tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+  }
+  ap.cent = cent;
+  ap.assign = assign;
+  ap.st = w.st;
+  ap.lim = wait_limit_ns();
+  ap.N = N;
+  ap.k = k;
+  const int kp = k <= 32 ? 32 : 64;
+  const size_t assign_smem = 1024 + 32768 + (size_t)4 * kp * 128;
+  auto assign_kernel = kp == 32 ? km_assign_kernel<32> : km_assign_kernel<64>;
   if (cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)assign_smem) !=
       cudaSuccess)
     return fail(VCA_ERR_CUDA, "vca_cluster_permute: cannot set shared-memory size");
-  const dim3 g_assign((N + 2 * kAssignThreads - 1) / (2 * kAssignThreads), BH);
+  const dim3 g_assign((N + 127) / 128, BH);
   const dim3 g_accum((N + kSegWarps * kSegTok - 1) / (kSegWarps * kSegTok), BH);
   const int nchunk = (N + kSortChunk - 1) / kSortChunk;
   // Every round: assign, stable counting sort by cluster (its scan also gives
   // the cluster sizes and starts), exact sums along the sorted order, update.
   // The last round's sort is the permutation the caller gets.
   for (int it = 0; it < iters; ++it) {
-    assign_kernel<<<g_assign, kAssignThreads, assign_smem, s>>>(V, cent, assign, N, k);
+    assign_kernel<<<g_assign, kAsgThreads, assign_smem, s>>>(ap);
     if ((rc = check_launch("km_assign_kernel"))) return rc;
     sort_count_kernel<<<dim3(nchunk, BH), 256, 0, s>>>(assign, w.ccount, N, k, nchunk);
     if ((rc = check_launch("sort_count_kernel"))) return rc;

@@ -117,3 +117,38 @@ def test_grouping_reports_values_outside_its_exact_range(bad, code):
     V[0, 1, 77, 5] = 2.0 ** 19
     vca.cluster_permute(V, w.k, 3, ws=ws)
     ws.check()
+
+
+@pytest.mark.parametrize("k", [1, 5, 32, 33, 64])
+def test_assignment_ties_and_near_ties(k):
+    # the assignment evaluates the defined distance only for the centroids a
+    # tensor-core estimate cannot rule out: centroids that tie exactly (the
+    # lower index must win), differ by one unit in the last place, or sit on
+    # either side of a token at the same distance must all reach the exact
+    # comparison, and the result must equal the oracle's full scan
+    w = W.shrink(W.WORKLOADS[2], H=2, N=777)
+    _, _, V = W.make_qkv(w, "cuda")
+    Vf = V.float().cpu().numpy()
+    rng = np.random.default_rng(11 + k)
+    init = np.empty((1, w.H, k, 128), dtype=np.float32)
+    for h in range(w.H):
+        idx = rng.choice(w.N, size=k, replace=False)
+        c = Vf[0, h, idx].copy()
+        if k >= 2:
+            c[1] = c[0]                                   # exact tie with centroid 0
+        if k >= 4:
+            c[3] = c[2]
+            c[3, 17] = np.nextafter(c[2, 17], np.float32(np.inf))   # one ulp apart
+        if k >= 6:
+            t = Vf[0, h, idx[4]]                          # a token between 4 and 5
+            c[4] = t
+            c[5] = t
+            c[4, 9] = t[9] + np.float32(0.25)
+            c[5, 9] = t[9] - np.float32(0.25)
+        init[0, h] = c
+    _, assign, _ = vca.cluster_permute(V, k, iters=1, init=torch.from_numpy(init).cuda())
+    torch.cuda.synchronize()
+    for h in range(w.H):
+        want = oracle.kmeans_assign(Vf[0, h], init[0, h])
+        got = assign[0, h].cpu().numpy()
+        assert np.array_equal(got, want), (h, np.argwhere(got != want)[:5].tolist())
