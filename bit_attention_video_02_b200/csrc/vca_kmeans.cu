@@ -108,8 +108,13 @@ struct AsgParams {
 // KP centroid slots (32 for k <= 32, else 64): two B matrices of KP rows, the
 // bf16 hi parts and the lo parts of the centroids, accumulated into the same
 // KP tensor-memory columns (column c = v.hi_c + v.lo_c, 256 products).
+// Persistent over one head: CTA x takes the head's 128-token tiles x, x + G,
+// x + 2G, ... (G = gridDim.x), so the centroid operand and the tensor memory are
+// set up once per CTA; each thread keeps its token's row in registers, so the
+// one V buffer takes the next tile's TMA copy while this tile is filtered and
+// its candidates evaluated.
 template <int KP>
-__global__ void __launch_bounds__(kAsgThreads, 4) km_assign_kernel(const __grid_constant__ AsgParams p) {
+__global__ void __launch_bounds__(kAsgThreads, 3) km_assign_kernel(const __grid_constant__ AsgParams p) {
   constexpr uint32_t kBChunk = KP * 128;   // bytes of one 64-channel chunk of a B matrix
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -120,16 +125,17 @@ __global__ void __launch_bounds__(kAsgThreads, 4) km_assign_kernel(const __grid_
   __shared__ int abort_s, never_s;
   __shared__ float nc_s[KP];
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int bh = blockIdx.y, tile = blockIdx.x, k = p.k;
+  const int bh = blockIdx.y, k = p.k, G = gridDim.x;
+  const int ntiles = (p.N + 127) / 128;
   if (tid == 0) {
     abort_s = 0;
     never_s = 0;
     mbar_init(&bar_full, 1);
     mbar_init(&bar_mma, 1);
     fence_barrier_init();
-    mbar_arrive_expect_tx(&bar_full, 32768);
-    tma_load_3d(sV, &p.tmV, &bar_full, 0, tile * 128, bh);
-    tma_load_3d(sV + 16384, &p.tmV, &bar_full, 64, tile * 128, bh);
+    mbar_arrive_expect_tx(&bar_full, 32768);   // the first tile (blockIdx.x < ntiles)
+    tma_load_3d(sV, &p.tmV, &bar_full, 0, blockIdx.x * 128, bh);
+    tma_load_3d(sV + 16384, &p.tmV, &bar_full, 64, blockIdx.x * 128, bh);
   }
   // B: thread pair (c, half) writes centroid c's channels 64 half .. +63 as bf16
   // hi and lo (row c of either matrix) in 16-byte units swizzled by the row
@@ -178,16 +184,22 @@ __global__ void __launch_bounds__(kAsgThreads, 4) km_assign_kernel(const __grid_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
-  bool issued = false;
-  if (warp == 0) {
-    // D[token][c] = sum over the 128 channels of v (hi_c + lo_c): 8 steps of 16
-    // channels against each matrix
-    issued = mbar_wait_warp(&bar_full, 0, &abort_s, p.st, p.lim, 500);
-    if (issued) {
+  const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+  const uint32_t idesc = instr_desc(kFmtBF16, kFmtBF16, 128, KP, 0, 0);
+  const uint64_t dA = smem_desc(smem_u32(sV), 16, 1024, kLayoutSW128);
+  const uint64_t dB = smem_desc(smem_u32(sB), 16, 1024, kLayoutSW128);
+  const float4* cb = reinterpret_cast<const float4*>(p.cent + (int64_t)bh * k * 128);
+  // for the exit after a failed wait: what may still be in flight
+  bool full_ok = true, mma_issued = false, mma_ok = true;
+  uint32_t ph = 0;
+  for (int i = 0, tile = blockIdx.x; tile < ntiles; ++i, tile += G) {
+    ph = (uint32_t)i & 1u;
+    full_ok = mbar_wait_warp(&bar_full, ph, &abort_s, p.st, p.lim, 500);
+    mma_issued = false;
+    if (warp == 0 && full_ok) {
+      // D[token][c] = sum over the 128 channels of v (hi_c + lo_c): 8 steps of 16
+      // channels against each matrix
       tc_fence_after();
-      const uint32_t idesc = instr_desc(kFmtBF16, kFmtBF16, 128, KP, 0, 0);
-      const uint64_t dA = smem_desc(smem_u32(sV), 16, 1024, kLayoutSW128);
-      const uint64_t dB = smem_desc(smem_u32(sB), 16, 1024, kLayoutSW128);
 #pragma unroll
       for (int s = 0; s < 16; ++s) {   // +32 bytes per step inside a 128-byte row, then the next chunk
         const int st = s & 7;
@@ -195,30 +207,37 @@ __global__ void __launch_bounds__(kAsgThreads, 4) km_assign_kernel(const __grid_
                       dB + (uint64_t)(((s >> 3) * 2 + (st >> 2)) * (kBChunk / 16) + (st & 3) * 2), idesc, s > 0);
       }
       tc_commit_w(&bar_mma);
+      mma_issued = true;
     }
-  }
-  // this thread's token: row tid of the tile (16-byte units swizzled by the
-  // row index), and |v|^2
-  bool ok = mbar_wait_warp(&bar_full, 0, &abort_s, p.st, p.lim, 501);
-  const uint8_t* vrow = sV + tid * 128;
-  const int vsw = tid & 7;
-  float nv = 0.0f;
-  if (ok) {
+    // this thread's token: row tid of the tile (16-byte units swizzled by the
+    // row index) into registers, and |v|^2
+    uint32_t vr[64];
+    float nv = 0.0f;
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
-      const uint4 x = *reinterpret_cast<const uint4*>(vrow + (u >> 3) * 16384 + (((u & 7) ^ vsw) << 4));
-      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        nv = fmaf(bf16_lo(w[e]), bf16_lo(w[e]), nv);
-        nv = fmaf(bf16_hi(w[e]), bf16_hi(w[e]), nv);
-      }
+      uint4 x = make_uint4(0u, 0u, 0u, 0u);
+      if (full_ok)
+        x = *reinterpret_cast<const uint4*>(sV + (u >> 3) * 16384 + tid * 128 + (((u & 7) ^ (tid & 7)) << 4));
+      vr[4 * u] = x.x;
+      vr[4 * u + 1] = x.y;
+      vr[4 * u + 2] = x.z;
+      vr[4 * u + 3] = x.w;
     }
-  }
-  ok = ok && mbar_wait_warp(&bar_mma, 0, &abort_s, p.st, p.lim, 502);
-  if (ok) {
+#pragma unroll
+    for (int w = 0; w < 64; ++w) {
+      nv = fmaf(bf16_lo(vr[w]), bf16_lo(vr[w]), nv);
+      nv = fmaf(bf16_hi(vr[w]), bf16_hi(vr[w]), nv);
+    }
+    mma_ok = full_ok && mbar_wait_warp(&bar_mma, ph, &abort_s, p.st, p.lim, 502);
+    // every row is in registers and the MMA has read the tile: the buffer may
+    // take the next tile (a failed wait anywhere stops every thread here)
+    if (__syncthreads_or(!mma_ok)) break;
     tc_fence_after();
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    if (tid == 0 && tile + G < ntiles) {
+      mbar_arrive_expect_tx(&bar_full, 32768);
+      tma_load_3d(sV, &p.tmV, &bar_full, 0, (tile + G) * 128, bh);
+      tma_load_3d(sV + 16384, &p.tmV, &bar_full, 64, (tile + G) * 128, bh);
+    }
     // pass 1: the smallest upper bound; pass 2: the candidates
     float best_ub = INFINITY;
     bool bad = !(fabsf(nv) < INFINITY);
@@ -248,9 +267,11 @@ __global__ void __launch_bounds__(kAsgThreads, 4) km_assign_kernel(const __grid_
         }
       }
     }
+    // every thread has read its row of D: the next tile's MMA may overwrite it
+    tc_fence_before();
+    __syncthreads();
     if (bad || !(best_ub < INFINITY)) cand = k == 64 ? ~0ull : (1ull << k) - 1;
     // the defined distance for the candidates, in increasing index
-    const float4* cb = reinterpret_cast<const float4*>(p.cent + (int64_t)bh * k * 128);
     int best = 0;
     float bd = 0.0f;
     bool first = true;
@@ -260,17 +281,16 @@ __global__ void __launch_bounds__(kAsgThreads, 4) km_assign_kernel(const __grid_
       const float4* mu = cb + c * 32;
       float acc = 0.0f;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {   // channels 8u .. 8u + 7
-        const uint4 x = *reinterpret_cast<const uint4*>(vrow + (u >> 3) * 16384 + (((u & 7) ^ vsw) << 4));
-        const float4 m0 = __ldg(mu + 2 * u), m1 = __ldg(mu + 2 * u + 1);
-        const float vv[8] = {bf16_lo(x.x), bf16_hi(x.x), bf16_lo(x.y), bf16_hi(x.y),
-                             bf16_lo(x.z), bf16_hi(x.z), bf16_lo(x.w), bf16_hi(x.w)};
-        const float mm[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float t = __fsub_rn(vv[e], mm[e]);
-          acc = __fmaf_rn(t, t, acc);
-        }
+      for (int q = 0; q < 32; ++q) {   // channels 4q .. 4q + 3
+        const float4 m = __ldg(mu + q);
+        float t = __fsub_rn(bf16_lo(vr[2 * q]), m.x);
+        acc = __fmaf_rn(t, t, acc);
+        t = __fsub_rn(bf16_hi(vr[2 * q]), m.y);
+        acc = __fmaf_rn(t, t, acc);
+        t = __fsub_rn(bf16_lo(vr[2 * q + 1]), m.z);
+        acc = __fmaf_rn(t, t, acc);
+        t = __fsub_rn(bf16_hi(vr[2 * q + 1]), m.w);
+        acc = __fmaf_rn(t, t, acc);
       }
       if (first || acc < bd) {
         bd = acc;
@@ -281,9 +301,9 @@ __global__ void __launch_bounds__(kAsgThreads, 4) km_assign_kernel(const __grid_
     const int n = tile * 128 + tid;
     if (n < p.N) p.assign[(int64_t)bh * p.N + n] = best;
   }
-  // nothing may be in flight into this CTA's memory when it exits
-  if (tid == 0 && !ok) mbar_wait_bounded(&bar_full, 0, &never_s, nullptr, p.lim, 503);
-  if (warp == 0 && issued && !ok) mbar_wait_warp(&bar_mma, 0, &never_s, nullptr, p.lim, 504);
+  // after a failed wait, nothing may still be in flight into this CTA's memory
+  if (tid == 0 && !full_ok) mbar_wait_bounded(&bar_full, ph, &never_s, nullptr, p.lim, 503);
+  if (warp == 0 && mma_issued && !mma_ok) mbar_wait_warp(&bar_mma, ph, &never_s, nullptr, p.lim, 504);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -535,7 +555,14 @@ static int cluster_permute_impl(const vca_bf16* V, int B, int H, int N, int d, i
   if (cudaFuncSetAttribute(assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)assign_smem) !=
       cudaSuccess)
     return fail(VCA_ERR_CUDA, "vca_cluster_permute: cannot set shared-memory size");
-  const dim3 g_assign((N + 127) / 128, BH);
+  // persistent over a head's tiles: about 3 CTAs per SM over the whole layer, so
+  // one wave (and at least one CTA per head)
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int ntiles = (N + 127) / 128;
+  int per_head = 3 * sms / BH;
+  per_head = per_head < 1 ? 1 : (per_head > ntiles ? ntiles : per_head);
+  const dim3 g_assign(per_head, BH);
   const dim3 g_accum((N + kSegWarps * kSegTok - 1) / (kSegWarps * kSegTok), BH);
   const int nchunk = (N + kSortChunk - 1) / kSortChunk;
   // Every round: assign, stable counting sort by cluster (its scan also gives
