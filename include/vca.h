@@ -120,7 +120,11 @@ size_t vca_cluster_permute_workspace_size(int B, int H, int N, int k);
  *   perm       [B][H][N] int32          (out)
  * 1 <= k <= VCA_MAX_CLUSTERS, 1 <= iters <= 64, |V| < 2^20: a value outside
  * that range records VCA_ERR_INVALID (VCA_ERR_NONFINITE for inf/NaN) in the
- * workspace status word (vca_check_status). */
+ * workspace status word (vca_check_status), as does a device wait that runs
+ * out (VCA_ERR_TIMEOUT).  All pointers 16-byte aligned, else VCA_ERR_INVALID.
+ * The assignment evaluates the distance above only for the centroids that a
+ * tensor-core estimate with a proven error bound cannot rule out; the result
+ * is the full scan's, bit for bit. */
 int vca_cluster_permute(const vca_bf16* V, int B, int H, int N, int d, int k, int iters,
                         const float* init_centroids, float* centroids, int32_t* assign,
                         int32_t* perm, void* ws, size_t ws_bytes, vca_stream_t stream);
