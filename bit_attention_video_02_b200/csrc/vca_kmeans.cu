@@ -17,8 +17,6 @@
 // (one fp64 division per centroid coordinate).  Then a stable counting sort:
 // per-chunk histograms, an exclusive scan in (cluster, chunk) order, and a
 // warp-synchronous ranked scatter.
-#include <mutex>
-
 #include "vca_device.cuh"
 #include "vca_host.h"
 
